@@ -1,0 +1,239 @@
+// C ABI of libspattn (declared in include/spattn.h): argument checks, tensor
+// maps, and the launch sequence of each pass.  No allocation happens here
+// except in spattn_plan (the plan's device lists and workspace).
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <new>
+
+#include "kernels.cuh"
+#include "plan.hpp"
+
+namespace spattn {
+int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P);
+void free_plan_device(spattn_plan_s* P);
+void canonical_pages(const spattn_plan_s& P, int32_t h, int64_t qb, std::vector<int32_t>& out);
+void transposed_qblocks(const spattn_plan_s& P, int32_t h, int64_t page, std::vector<int32_t>& out);
+int64_t bsa_pairs(const spattn_plan_s& P);
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [rows_per_bh, head_dim] bf16 matrices stacked over batch*heads; boxes of
+// 16 rows x 64 columns, 128-byte swizzle (the layout the MMA descriptors
+// expect).  Rows past the end of a (batch, head) read as zeros.
+bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(head_dim) * 2 * rows};
+  cuuint32_t box[3] = {64, 16, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_plan_device(const spattn_plan_s* P) {
+  if (P->device < 0) return SPATTN_ERR_CUDA;  // host-only plan (no device when it was built)
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPATTN_ERR_CUDA;
+  return dev == P->device ? SPATTN_OK : SPATTN_ERR_INVALID_ARG;
+}
+
+TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots) {
+  TileArgs a;
+  a.work = w.d_work;
+  a.pages = w.d_pages;
+  a.masks = w.d_masks;
+  a.n_work = w.n_work;
+  a.own_slots = own_slots;
+  a.col_slots = col_slots;
+  a.scale = P->scale;
+  a.err = P->d_err;
+  return a;
+}
+
+}  // namespace
+}  // namespace spattn
+
+using namespace spattn;
+
+extern "C" {
+
+int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_plan_t* out) {
+  if (!out) return SPATTN_ERR_INVALID_ARG;
+  *out = nullptr;
+  spattn_plan_s* P = nullptr;
+  try {
+    P = new spattn_plan_s();
+    const int st = build_plan(layout, graph, P);
+    if (st != SPATTN_OK) {
+      free_plan_device(P);
+      delete P;
+      return st;
+    }
+  } catch (const std::bad_alloc&) {
+    if (P) {
+      free_plan_device(P);
+      delete P;
+    }
+    return SPATTN_ERR_OOM;
+  }
+  *out = P;
+  return SPATTN_OK;
+}
+
+int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, void* o, float* lse, void* stream) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return SPATTN_ERR_INVALID_ARG;
+  const int D = plan->head_dim;
+  const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, D, plan->q.slots, bh) || !make_map(&tk, k, D, plan->k.slots, bh) ||
+      !make_map(&tv, v, D, plan->k.slots, bh))
+    return SPATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* O = static_cast<__nv_bfloat16*>(o);
+  cudaError_t e = launch_fwd(D, tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), O, lse, s);
+  if (e == cudaSuccess)
+    e = launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots, O,
+                    nullptr, lse, s);
+  return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
+}
+
+int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* d_o,
+               spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !aligned16(d_o) ||
+      !aligned16(dq) || !aligned16(dk) || !aligned16(dv))
+    return SPATTN_ERR_INVALID_ARG;
+  const int D = plan->head_dim;
+  const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_map(&tq, q, D, plan->q.slots, bh) || !make_map(&tk, k, D, plan->k.slots, bh) ||
+      !make_map(&tv, v, D, plan->k.slots, bh) || !make_map(&tdo, d_o, D, plan->q.slots, bh))
+    return SPATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* dQ = static_cast<__nv_bfloat16*>(dq);
+  auto* dK = static_cast<__nv_bfloat16*>(dk);
+  auto* dV = static_cast<__nv_bfloat16*>(dv);
+  cudaError_t e = launch_delta(D, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o),
+                               plan->d_delta, bh * plan->q.slots, s);
+  if (e == cudaSuccess)
+    e = launch_dkdv(D, tk, tv, tq, tdo, tile_args(plan, plan->wk, plan->k.slots, plan->q.slots), lse, plan->d_delta,
+                    dK, dV, s);
+  if (e == cudaSuccess)
+    e = launch_dq(D, tq, tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, plan->d_delta,
+                  dQ, s);
+  if (e == cudaSuccess)
+    e = launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots, dK,
+                    dV, nullptr, s);
+  if (e == cudaSuccess)
+    e = launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots, dQ,
+                    nullptr, nullptr, s);
+  return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
+}
+
+int spattn_check(spattn_plan_t plan, void* stream) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  if (plan->device < 0) return SPATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SPATTN_ERR_CUDA;
+  int h = 0;
+  if (cudaMemcpy(&h, plan->d_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SPATTN_ERR_CUDA;
+  if (h == 0) return SPATTN_OK;
+  if (cudaMemset(plan->d_err, 0, sizeof(int)) != cudaSuccess) return SPATTN_ERR_CUDA;
+  return h == 1 ? SPATTN_ERR_TIMEOUT : SPATTN_ERR_DEVICE;
+}
+
+int spattn_plan_stats(spattn_plan_t plan, spattn_stats* s) {
+  if (!plan || !s) return SPATTN_ERR_INVALID_ARG;
+  if (plan->bsa_pairs < 0) plan->bsa_pairs = bsa_pairs(*plan);
+  std::memset(s, 0, sizeof(*s));
+  s->useful_pairs = plan->useful_pairs;
+  s->physical_pairs_fwd = plan->wq.physical_pairs * plan->batch;
+  s->physical_pairs_dq = plan->wq.physical_pairs * plan->batch;
+  s->physical_pairs_dkdv = plan->wk.physical_pairs * plan->batch;
+  s->bsa_pairs = plan->bsa_pairs;
+  s->n_work_fwd = plan->wq.n_work;
+  s->n_work_dkdv = plan->wk.n_work;
+  s->n_entries_fwd = static_cast<int64_t>(plan->wq.pages.size());
+  s->n_entries_dkdv = static_cast<int64_t>(plan->wk.pages.size());
+  s->device_bytes = plan->device_bytes;
+  s->plan_ms = plan->plan_ms;
+  return SPATTN_OK;
+}
+
+int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const int32_t** pages, int64_t* n) {
+  if (!plan || !pages || !n || head < 0 || head >= plan->heads || qblock < 0 ||
+      qblock >= (plan->q.slots + kBlockRows - 1) / kBlockRows)
+    return SPATTN_ERR_INVALID_ARG;
+  canonical_pages(*plan, head, qblock, plan->scratch);
+  *pages = plan->scratch.data();
+  *n = static_cast<int64_t>(plan->scratch.size());
+  return SPATTN_OK;
+}
+
+int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const int32_t** qblocks, int64_t* n) {
+  if (!plan || !qblocks || !n || head < 0 || head >= plan->heads || page < 0 || page >= plan->k.n_pages)
+    return SPATTN_ERR_INVALID_ARG;
+  transposed_qblocks(*plan, head, page, plan->scratch);
+  *qblocks = plan->scratch.data();
+  *n = static_cast<int64_t>(plan->scratch.size());
+  return SPATTN_OK;
+}
+
+int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work, const int32_t** pages,
+                     const uint64_t** masks, int64_t* n_entries) {
+  if (!plan || !work || !n_work || !pages || !masks || !n_entries || (which != 0 && which != 1))
+    return SPATTN_ERR_INVALID_ARG;
+  const WorkList& w = which == 0 ? plan->wq : plan->wk;
+  *work = w.work.data();
+  *n_work = w.n_work;
+  *pages = w.pages.data();
+  *masks = w.masks.data();
+  *n_entries = static_cast<int64_t>(w.pages.size());
+  return SPATTN_OK;
+}
+
+void spattn_plan_destroy(spattn_plan_t plan) {
+  if (!plan) return;
+  free_plan_device(plan);
+  delete plan;
+}
+
+const char* spattn_status_string(int status) {
+  switch (status) {
+    case SPATTN_OK: return "ok";
+    case SPATTN_ERR_INVALID_ARG: return "invalid argument";
+    case SPATTN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SPATTN_ERR_OOM: return "out of memory";
+    case SPATTN_ERR_CUDA: return "CUDA runtime error";
+    case SPATTN_ERR_TIMEOUT: return "device-side wait timed out";
+    case SPATTN_ERR_DEVICE: return "device rejected a work item";
+    default: return "unknown status";
+  }
+}
+
+}  // extern "C"

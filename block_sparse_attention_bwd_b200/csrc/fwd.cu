@@ -1,0 +1,334 @@
+// K1: forward attention over packed pages, and K5: fill of page-sized holes.
+//
+// Method (KPage abstract, "KPage: block-sparse attention for partially
+// occupied 3D blocks", zhuanzhiai.com, abstract paragraph): valid 16-row K/V
+// pages are packed into large tiles while they are loaded, with no compacted
+// copy in HBM, and masking stays exact.  The softmax is the online
+// (streaming) form used by FlashAttention-style kernels.
+//
+// One CTA runs one query-owned work item: up to 8 query pages (128 rows,
+// TMEM lanes) against its list of key pages, 8 pages (128 columns) per step.
+//   warp 0      TMA producer: query pages once, then K and V pages of each
+//               step into an NS-deep ring, one 16-row box per page and
+//               64-column chunk (gathered straight from [B,H,S,D] memory);
+//   warp 1      allocates TMEM and issues tcgen05 MMAs from one thread:
+//               S_b = Q K^T into one of two TMEM buffers, then O += P V with
+//               P read from TMEM (bf16, written over S_b by the softmax);
+//   warps 4..7  one tile row per thread: exact mask from the step's page
+//               masks, running max with lazy rescaling, P in bf16 to TMEM,
+//               and the epilogue (O / l, LSE in natural log).
+// S is double-buffered, so the MMA of step c+1 overlaps the softmax of c.
+#include "kernels.cuh"
+#include "tile.cuh"
+
+namespace spattn {
+namespace {
+
+using namespace dev;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kNch = D / 64;                      // 64-column chunks
+  static constexpr int kTile = kNch * kChunkBytes;         // one 128-row operand
+  static constexpr int kStages = (D == 128) ? 2 : 4;       // K/V ring depth
+  static constexpr int kSmem = kTile * (1 + 2 * kStages) + 1024 + 256;
+};
+
+// Rescale O only when the running max grows by more than 2^8 (log2 units):
+// P stays below 256 and the final O / l is unchanged.
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+               const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ work,
+               const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
+               __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
+               int* err) {
+  using C = FwdCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::kTile;  // stage s: K at sKV + 2*s*kTile, V right after
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kTile * (1 + 2 * NS));
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + NS;
+  uint64_t* kv_empty = v_full + NS;
+  uint64_t* s_full = kv_empty + NS;  // [2]
+  uint64_t* p_full = s_full + 2;     // [2]
+  uint64_t* o_done = p_full + 2;
+  uint64_t* drain = o_done + 1;
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
+  const Abort ab{abort_flag, err};
+
+  const Work wk = load_work(work, blockIdx.x);
+  const int n_cols = wk.e1 - wk.e0;
+  const int n_steps = (n_cols + kStepPages - 1) / kStepPages;
+  const int warp = warp_id(), lane = lane_id();
+
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    mbar_init(q_full, 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(drain, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tslot, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tslot;
+  const uint32_t tO = tmem + 256;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- producer ----------------
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_arrive_expect_tx(q_full, wk.n_own * C::kNch * 2048);
+      for (int p = 0; p < wk.n_own; ++p)
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sQ + c * kChunkBytes + p * 2048, &tm_q, c * 64, wk.own_page(p) * 16, wk.bh, q_full);
+      int issued = 0;
+      for (int st = 0; st < n_steps; ++st) {
+        const int s = st % NS;
+        if (st >= NS && !mbar_wait(&kv_empty[s], ((st / NS) - 1) & 1, ab)) break;
+        const int n = min(kStepPages, n_cols - st * kStepPages);
+        uint8_t* kd = sKV + 2 * s * C::kTile;
+        uint8_t* vd = kd + C::kTile;
+        const int32_t* pg = col_pages + wk.e0 + st * kStepPages;
+        mbar_arrive_expect_tx(&k_full[s], n * C::kNch * 2048);
+        for (int j = 0; j < n; ++j) {
+          const int row = __ldg(pg + j) * 16;
+          for (int c = 0; c < C::kNch; ++c) tma_load_3d(kd + c * kChunkBytes + j * 2048, &tm_k, c * 64, row, wk.bh, &k_full[s]);
+        }
+        mbar_arrive_expect_tx(&v_full[s], n * C::kNch * 2048);
+        for (int j = 0; j < n; ++j) {
+          const int row = __ldg(pg + j) * 16;
+          for (int c = 0; c < C::kNch; ++c) tma_load_3d(vd + c * kChunkBytes + j * 2048, &tm_v, c * 64, row, wk.bh, &v_full[s]);
+        }
+        issued = st + 1;
+      }
+      // make sure no copy is still landing in shared memory when the CTA exits
+      for (int st = max(0, issued - NS); st < issued; ++st) {
+        mbar_wait_drain(&k_full[st % NS], (st / NS) & 1);
+        mbar_wait_drain(&v_full[st % NS], (st / NS) & 1);
+      }
+      mbar_wait_drain(q_full, 0);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      const uint32_t q_addr = smem_u32(sQ);
+      const uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+      bool ok = mbar_wait(q_full, 0, ab);
+      tc_fence_after();
+      auto issue_pv = [&](int st) -> bool {
+        const int b = st & 1, s = st % NS;
+        if (!mbar_wait(&p_full[b], (st >> 1) & 1, ab)) return false;
+        if (!mbar_wait(&v_full[s], (st / NS) & 1, ab)) return false;
+        tc_fence_after();
+        const int n = min(kStepPages, n_cols - st * kStepPages);
+        const uint32_t v_addr = smem_u32(sKV + 2 * s * C::kTile + C::kTile);
+        for (int j = 0; j < n; ++j)
+          umma_ts(tO, tmem + 128 * b + 8 * j, sdesc_sw128(v_addr + j * 2048, kChunkBytes, 1024), idesc_pv,
+                  (st > 0 || j > 0) ? 1u : 0u);
+        umma_commit(&kv_empty[s]);
+        umma_commit(o_done);
+        return true;
+      };
+      for (int st = 0; ok && st < n_steps; ++st) {
+        const int s = st % NS, b = st & 1;
+        if (!mbar_wait(&k_full[s], (st / NS) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int n = min(kStepPages, n_cols - st * kStepPages);
+        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+        const uint32_t k_addr = smem_u32(sKV + 2 * s * C::kTile);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
+          umma_ss(tmem + 128 * b, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[b]);
+        if (st >= 1 && !issue_pv(st - 1)) ok = false;
+      }
+      if (ok && n_steps > 0) issue_pv(n_steps - 1);
+      umma_commit(drain);
+      mbar_wait_drain(drain, 0);
+    }
+  } else if (warp >= 4) {
+    // ---------------- softmax + epilogue (one row per thread) ----------------
+    const int q4 = warp - 4;
+    const int row = q4 * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t code = wk.row_code(row);
+    const int seg = code < 4 ? static_cast<int>(code) : -1;
+    float m_used = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int st = 0; st < n_steps; ++st) {
+      const int b = st & 1;
+      const int n = min(kStepPages, n_cols - st * kStepPages);
+      const int N = 16 * n;
+      uint32_t mw[4];
+      step_masks(col_masks, wk.e0 + st * kStepPages, n, seg, mw);
+      ok = mbar_wait(&s_full[b], (st >> 1) & 1, ab);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc)
+        if (pc * 32 < N) tmem_ld32(tmem + 128 * b + lane_off + pc * 32, sr[pc]);
+      tmem_wait_ld();
+      float mx = -INFINITY;
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const bool on = (pc * 32 < N) && ((mw[pc] >> i) & 1u);
+          const float x = on ? __uint_as_float(sr[pc][i]) * sl2 : -INFINITY;
+          sr[pc][i] = __float_as_uint(x);
+          mx = fmaxf(mx, x);
+        }
+      }
+      const bool resc = mx > m_used + kRescaleThreshold;
+      const float m_new = resc ? mx : m_used;
+      const float alpha = resc ? ex2(m_used - m_new) : 1.0f;
+      if (st > 0 && __any_sync(0xffffffffu, resc)) {
+        // O holds steps < st: wait for the last PV, then rescale this warp's rows
+        ok = mbar_wait(o_done, (st - 1) & 1, ab);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll
+        for (int pc = 0; pc < D / 32; ++pc) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + pc * 32, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(tO + lane_off + pc * 32, r);
+        }
+      }
+      l *= alpha;
+      m_used = m_new;
+      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+      float lsum = 0.f;
+#pragma unroll
+      for (int pc = 0; pc < 4; ++pc) {
+        if (pc * 32 < N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float p0 = ex2(__uint_as_float(sr[pc][2 * i]) - mu);
+            const float p1 = ex2(__uint_as_float(sr[pc][2 * i + 1]) - mu);
+            lsum += p0 + p1;
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tmem + 128 * b + lane_off + pc * 16, pk);
+        }
+      }
+      l += lsum;
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&p_full[b]);
+    }
+    if (ok && n_steps > 0) {
+      ok = mbar_wait(o_done, (n_steps - 1) & 1, ab);
+      ok = __all_sync(0xffffffffu, ok);
+      tc_fence_after();
+    }
+    if (ok) {
+      const bool owned = code != 15u && row < 16 * wk.n_own;
+      const int64_t slot = owned ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+      const bool write = owned && slot < q_slots;
+      const bool empty = !(l > 0.f);
+      const float inv = empty ? 0.f : 1.0f / l;
+      __nv_bfloat16* dst = out_o + (static_cast<int64_t>(wk.bh) * q_slots + slot) * D;
+#pragma unroll
+      for (int pc = 0; pc < D / 32; ++pc) {
+        uint32_t r[32] = {};
+        if (n_steps > 0) {
+          tmem_ld32(tO + lane_off + pc * 32, r);
+          tmem_wait_ld();
+        }
+        if (write) store_row32(dst + pc * 32, r, inv, empty || n_steps == 0);
+      }
+      if (write) out_lse[static_cast<int64_t>(wk.bh) * q_slots + slot] = empty ? -INFINITY : (m_used + lg2(l)) * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// Zero 16-row pages that hold no valid slot; LSE rows (if given) get -inf.
+__global__ void fill_kernel(const int32_t* __restrict__ pages, int64_t n_bh, int64_t slots, int head_dim,
+                            __nv_bfloat16* __restrict__ t0, __nv_bfloat16* __restrict__ t1, float* __restrict__ lse) {
+  const int64_t page = pages[blockIdx.x];
+  const int vec_per_row = head_dim / 8;  // 16-byte vectors
+  for (int64_t bh = blockIdx.y; bh < n_bh; bh += gridDim.y) {
+    for (int i = threadIdx.x; i < 16 * vec_per_row; i += blockDim.x) {
+      const int r = i / vec_per_row, c = i % vec_per_row;
+      const int64_t slot = page * 16 + r;
+      if (slot >= slots) continue;
+      const int64_t off = (bh * slots + slot) * head_dim + c * 8;
+      if (t0) *reinterpret_cast<uint4*>(t0 + off) = make_uint4(0, 0, 0, 0);
+      if (t1) *reinterpret_cast<uint4*>(t1 + off) = make_uint4(0, 0, 0, 0);
+    }
+    if (lse && threadIdx.x < 16) {
+      const int64_t slot = page * 16 + threadIdx.x;
+      if (slot < slots) lse[bh * slots + slot] = -INFINITY;
+    }
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TileArgs& a,
+                         __nv_bfloat16* o, float* lse, cudaStream_t st) {
+  using C = FwdCfg<D>;
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  if (a.n_work == 0) return cudaSuccess;
+  fwd_kernel<D><<<static_cast<unsigned>(a.n_work), 256, C::kSmem, st>>>(
+      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const TileArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t st) {
+  return head_dim == 128 ? launch_fwd_t<128>(tq, tk, tv, a, o, lse, st) : launch_fwd_t<64>(tq, tk, tv, a, o, lse, st);
+}
+
+cudaError_t launch_fill(int head_dim, const int32_t* pages, int64_t n_pages, int64_t bh, int64_t slots,
+                        __nv_bfloat16* t0, __nv_bfloat16* t1, float* lse, cudaStream_t st) {
+  if (n_pages == 0 || bh == 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>(n_pages), static_cast<unsigned>(bh < 65535 ? bh : 65535));
+  fill_kernel<<<grid, 128, 0, st>>>(pages, bh, slots, head_dim, t0, t1, lse);
+  return cudaGetLastError();
+}
+
+}  // namespace spattn

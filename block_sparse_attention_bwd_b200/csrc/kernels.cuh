@@ -1,0 +1,45 @@
+// Kernel launchers shared by the C ABI (api.cpp) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace spattn {
+
+// Everything one attention launch needs besides its tensor maps.
+struct TileArgs {
+  const int32_t* work = nullptr;    // n_work x 32 words (see spattn_plan_work)
+  const int32_t* pages = nullptr;   // column page ids
+  const uint64_t* masks = nullptr;  // 4 x 16-bit row masks per entry
+  int64_t n_work = 0;
+  int64_t own_slots = 0;            // rows per (batch, head) of the owned side
+  int64_t col_slots = 0;            // rows per (batch, head) of the column side
+  float scale = 0.f;                // softmax scale
+  int* err = nullptr;               // device error word
+};
+
+// K1: O, LSE for every query-owned work item.
+cudaError_t launch_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const TileArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t st);
+
+// K2: delta[row] = sum_d dO[row, d] * O[row, d] over rows = batch*heads*q_slots.
+cudaError_t launch_delta(int head_dim, const __nv_bfloat16* o, const __nv_bfloat16* d_o, float* delta,
+                         int64_t rows, cudaStream_t st);
+
+// K3: dK, dV for every key-owned work item.
+cudaError_t launch_dkdv(int head_dim, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
+                        const CUtensorMap& tdo, const TileArgs& a, const float* lse, const float* delta,
+                        __nv_bfloat16* dk, __nv_bfloat16* dv, cudaStream_t st);
+
+// K4: dQ for every query-owned work item.
+cudaError_t launch_dq(int head_dim, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
+                      const CUtensorMap& tv, const TileArgs& a, const float* lse, const float* delta,
+                      __nv_bfloat16* dq, cudaStream_t st);
+
+// K5: zero the rows of pages that hold no valid slot (and LSE = -inf).
+cudaError_t launch_fill(int head_dim, const int32_t* pages, int64_t n_pages, int64_t bh, int64_t slots,
+                        __nv_bfloat16* t0, __nv_bfloat16* t1, float* lse, cudaStream_t st);
+
+}  // namespace spattn

@@ -1,0 +1,77 @@
+// Device-side helpers shared by the attention kernels: work-item decode,
+// per-row masks of one 128-column step, smem layout constants.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace spattn {
+namespace dev {
+
+constexpr int kRows = 128;              // rows of an owned tile (TMEM lanes)
+constexpr int kStepPages = 8;           // column pages per step
+constexpr int kChunkBytes = 128 * 128;  // one 64-column chunk of a 128-row operand
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// Work item words (see spattn_plan_work in include/spattn.h).
+struct Work {
+  int bh, n_own, e0, e1;
+  const int32_t* w;
+  __device__ __forceinline__ int own_page(int i) const { return w[4 + i]; }
+  __device__ __forceinline__ uint32_t row_code(int r) const {
+    return (static_cast<uint32_t>(w[12 + (r >> 3)]) >> (4 * (r & 7))) & 0xFu;
+  }
+};
+
+__device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {
+  Work x;
+  x.w = work + idx * 32;
+  x.bh = x.w[0];
+  x.n_own = x.w[1];
+  x.e0 = x.w[2];
+  x.e1 = x.w[3];
+  return x;
+}
+
+// Row mask of one step: bit c of word c/32 <=> column c of the step may be
+// attended by this row.  `seg` < 0 gives an all-zero mask.
+__device__ __forceinline__ void step_masks(const uint64_t* __restrict__ masks, int first, int n, int seg,
+                                           uint32_t (&mw)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) mw[i] = 0u;
+  if (seg < 0) return;
+#pragma unroll
+  for (int j = 0; j < kStepPages; ++j) {
+    if (j < n) {
+      const uint32_t bits = static_cast<uint32_t>(__ldg(masks + first + j) >> (16 * seg)) & 0xFFFFu;
+      mw[j >> 1] |= bits << (16 * (j & 1));
+    }
+  }
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Store 32 fp32 values (times `mul`) of one row as bf16 to global memory.
+__device__ __forceinline__ void store_row32(__nv_bfloat16* dst, const uint32_t (&r)[32], float mul, bool zero) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float a = zero ? 0.f : __uint_as_float(r[2 * i]) * mul;
+    const float b = zero ? 0.f : __uint_as_float(r[2 * i + 1]) * mul;
+    pk[i] = pack_bf16(a, b);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+}
+
+}  // namespace dev
+}  // namespace spattn

@@ -1,0 +1,149 @@
+/*
+ * spattn — exact block-sparse softmax attention (forward and backward) for
+ * token layouts whose logical blocks are only partly occupied, on NVIDIA
+ * B200 (sm_100a).
+ *
+ * Problem statement: the KPage abstract ("KPage: block-sparse attention for
+ * partially occupied 3D blocks", zhuanzhiai.com, abstract paragraph).  A
+ * sparse graph over logical blocks of a 3D video token layout decides which
+ * query tokens may attend which key tokens; edge blocks of the T x H x W
+ * latent grid hold padded rows.  The method packs valid 16-row K/V pages
+ * into large tiles while loading, keeps exact per-row masking, and owns the
+ * K/V side in the backward pass so the sparse graph is preserved exactly in
+ * forward and backward.
+ *
+ * Data model
+ *   - A slot is one row of Q (or K/V).  q_group[i] >= 0 is the query group of
+ *     slot i; -1 marks a padded slot that is never a query.  kv_group[j] is
+ *     the same for keys.
+ *   - The graph is a CSR over (head, query group): entries
+ *     kv_groups[row_ptr[r] .. row_ptr[r+1]) with r = head * n_q_groups + a
+ *     are the key groups that query group a may attend in that head.  The
+ *     same graph serves every batch index.  Duplicate entries are allowed.
+ *   - Query slot i may attend key slot j in head h iff both are valid and
+ *     kv_group[j] is listed for q_group[i].
+ *   - A page is 16 consecutive slots; a Q block is 64 consecutive query
+ *     slots.
+ *
+ * Tensors (all device pointers, owned by the caller)
+ *   Q, O, dO, dQ : bf16 [batch, heads, q_slots, head_dim], contiguous
+ *   K, V, dK, dV : bf16 [batch, heads, kv_slots, head_dim], contiguous
+ *   LSE          : fp32 [batch, heads, q_slots], natural log of
+ *                  sum_j exp(scale * q_i . k_j) over the allowed keys.
+ *   Every pointer must be 16-byte aligned.  head_dim is 64 or 128.
+ *   Padded input rows may hold any finite values; outputs on padded or
+ *   attention-free query rows are O = 0, LSE = -inf, dQ = 0, and on padded
+ *   key rows dK = dV = 0.
+ *
+ * Errors: every call returns an SPATTN_* status; nothing throws across the
+ * ABI.  fwd/bwd are asynchronous on `stream` (a cudaStream_t, NULL = the
+ * legacy default stream) and launch nothing when an argument is rejected.
+ * Kernels never trap: a device-side wait that exceeds its deadline records an
+ * error in the plan, which spattn_check() reports.  A plan must not be used
+ * by two streams at the same time (the backward workspace is per plan).
+ */
+#ifndef SPATTN_H_
+#define SPATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum spattn_status {
+  SPATTN_OK = 0,
+  SPATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad group id */
+  SPATTN_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, slots beyond int32 rows, ... */
+  SPATTN_ERR_OOM = 3,         /* host or device allocation failed in spattn_plan */
+  SPATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed */
+  SPATTN_ERR_TIMEOUT = 5,     /* a kernel gave up on a device-side wait */
+  SPATTN_ERR_DEVICE = 6       /* a kernel rejected its work item */
+};
+
+typedef struct spattn_plan_s* spattn_plan_t; /* opaque, owned by the library */
+
+typedef struct {
+  int32_t batch, heads, head_dim; /* head_dim in {64, 128} */
+  int64_t q_slots, kv_slots;      /* >= 1 each; any length (ragged tails allowed) */
+  const int32_t* q_group;         /* host [q_slots], -1 = padded */
+  const int32_t* kv_group;        /* host [kv_slots], -1 = padded */
+  int32_t n_q_groups, n_kv_groups;
+  float scale;                    /* softmax scale; 0 selects 1/sqrt(head_dim) */
+} spattn_layout;
+
+typedef struct {
+  const int64_t* row_ptr;   /* host [heads * n_q_groups + 1], non-decreasing, row_ptr[0] = 0 */
+  const int32_t* kv_groups; /* host [row_ptr[heads * n_q_groups]], values in [0, n_kv_groups) */
+} spattn_graph;
+
+typedef struct {
+  int64_t useful_pairs;          /* allowed (query slot, key slot) pairs, all batches and heads */
+  int64_t physical_pairs_fwd;    /* pairs computed by the forward tiles (128 rows x 16 per page) */
+  int64_t physical_pairs_dkdv;   /* pairs computed by the dK/dV tiles */
+  int64_t physical_pairs_dq;     /* pairs computed by the dQ tiles */
+  int64_t bsa_pairs;             /* 64x64 x number of (Q block, K block) pairs with any allowed pair */
+  int64_t n_work_fwd;            /* forward / dQ work items (all batches) */
+  int64_t n_work_dkdv;           /* dK/dV work items (all batches) */
+  int64_t n_entries_fwd;         /* (work item, K page) entries of one batch */
+  int64_t n_entries_dkdv;        /* (work item, Q page) entries of one batch */
+  int64_t device_bytes;          /* device memory held by the plan */
+  double plan_ms;                /* host time spent in spattn_plan */
+} spattn_stats;
+
+/* Build a plan: validate layout and graph, find valid 16-row pages, pack
+ * owned tiles, and build the per-tile page lists and masks for the forward /
+ * dQ pass (query-owned) and the dK/dV pass (key-owned).  Host arrays are
+ * copied and may be freed afterwards.  Device lists are allocated on the
+ * current device with cudaMalloc and owned by the plan.  On a machine with no
+ * usable CUDA device the plan is built on the host only: the inspection
+ * calls (stats, pages, qblocks, work) work and spattn_fwd / spattn_bwd /
+ * spattn_check return SPATTN_ERR_CUDA. */
+int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_plan_t* out);
+
+/* Forward: O and LSE for every query slot of every (batch, head). */
+int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, void* o, float* lse,
+               void* stream);
+
+/* Backward: dQ, dK, dV given O and LSE from spattn_fwd and the loss
+ * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O). */
+int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* d_o,
+               spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream);
+
+/* Synchronise `stream` and report (then clear) any device-side error the
+ * plan's kernels recorded: SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_DEVICE. */
+int spattn_check(spattn_plan_t plan, void* stream);
+
+int spattn_plan_stats(spattn_plan_t plan, spattn_stats* stats);
+
+/* Canonical page list of (head, Q block): ascending pages holding at least
+ * one key that some query of the block may attend.  *pages points into a
+ * plan-owned buffer that stays valid until the next call on this plan. */
+int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const int32_t** pages, int64_t* n);
+
+/* Transposed list of (head, page): ascending Q blocks whose canonical list
+ * holds the page.  Same buffer rules as spattn_plan_pages. */
+int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const int32_t** qblocks, int64_t* n);
+
+/* Host copy of a work list, for inspection and tests.  which = 0: query-owned
+ * (forward and dQ), 1: key-owned (dK/dV).  Each work item is 32 int32 words:
+ *   [0] batch*heads + head   [1] owned page count n (<= 8)
+ *   [2] first entry          [3] end entry (into pages/masks)
+ *   [4..11] owned page ids   [12..27] 128 row codes, 4 bits each, row r in
+ *   word 12 + r/8 at bit 4*(r%8): 0..3 = segment, 14 = owned row with no
+ *   segment (padded), 15 = row not written by this item.
+ * pages[e] is a page id of the other side; masks[e] holds four 16-bit row
+ * masks over that page, one per segment (segment s in bits 16s..16s+15).
+ * Entries are shared by all batch indices. */
+int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work,
+                     const int32_t** pages, const uint64_t** masks, int64_t* n_entries);
+
+void spattn_plan_destroy(spattn_plan_t plan);
+
+const char* spattn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPATTN_H_ */

@@ -11,3 +11,10 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: large CPU work (still run by default)")
+
+
+def pytest_sessionstart(session):
+    """Build libspattn.so in-tree if it is missing or older than its sources."""
+    from block_sparse_attention_bwd_b200 import _build
+
+    _build.build()

@@ -1,0 +1,152 @@
+"""Planner (C-ABI, host side) against the oracle: canonical page lists and
+their transposes bit for bit, useful-pair counts exactly, and the coverage
+invariant of both work lists (every allowed pair computed by exactly one
+owned row of exactly one work item, and nothing else)."""
+
+import numpy as np
+import pytest
+
+import block_sparse_attention_bwd_b200 as sp
+import oracle
+from workloads import configs as W
+
+TINY = ["tiny", "tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey"]
+
+
+def _allowed(p, h):
+    return oracle.allowed_groups(p.row_ptr, p.kv_groups, p.n_q_groups, p.n_kv_groups, h)
+
+
+@pytest.mark.parametrize("name", TINY)
+def test_page_lists_bit_exact_tiny(name):
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p)
+    for h in range(p.heads):
+        A = _allowed(p, h)
+        for qb in range(-(-p.q_slots // 64)):
+            got = pl.pages(h, qb)
+            exp = oracle.canonical_pages(p.q_group, p.kv_group, A, qb)
+            assert got.dtype == np.int32 and np.array_equal(got, exp), (h, qb)
+        for pg in range(-(-p.kv_slots // 16)):
+            assert np.array_equal(pl.qblocks(h, pg), oracle.transposed_qblocks(p.q_group, p.kv_group, A, pg)), (h, pg)
+
+
+@pytest.mark.parametrize("name", TINY)
+def test_pair_counts_tiny(name):
+    p = W.make_problem(name)
+    for batch in (1, 2):
+        pl = sp.Plan.from_problem(p, batch=batch)
+        st = pl.stats()
+        brute = sum(oracle.useful_pairs_bruteforce(p.q_group, p.kv_group, _allowed(p, h)) for h in range(p.heads))
+        assert st["useful_pairs"] == brute * batch
+        bsa = sum(oracle.bsa_physical_pairs(p.q_group, p.kv_group, _allowed(p, h)) for h in range(p.heads))
+        assert st["bsa_pairs"] == bsa * batch
+        assert st["physical_pairs_fwd"] >= st["useful_pairs"]
+        assert st["physical_pairs_dkdv"] >= st["useful_pairs"]
+
+
+def _codes(w):
+    words = w[12:28].astype(np.int64) & 0xFFFFFFFF
+    return np.array([(words[r // 8] >> (4 * (r % 8))) & 0xF for r in range(128)])
+
+
+def _covered(p, pl, which, head_filter=None, row_filter=None):
+    """Pairs (own slot, column slot) per head produced by the work list, with multiplicity."""
+    work, pages, masks = pl.work(which)
+    own_group = p.q_group if which == 0 else p.kv_group
+    col_slots = p.kv_slots if which == 0 else p.q_slots
+    pairs = {}
+    owned = {}
+    bits16 = np.arange(16, dtype=np.uint64)
+    for w in work:
+        bh = int(w[0])
+        if bh >= p.heads:
+            continue  # batch copies repeat the same lists
+        h = bh
+        if head_filter is not None and h not in head_filter:
+            continue
+        n_own, e0, e1 = int(w[1]), int(w[2]), int(w[3])
+        assert 1 <= n_own <= 8 and 0 <= e0 <= e1 <= pages.size
+        codes = _codes(w)
+        pg = pages[e0:e1].astype(np.int64)
+        mk = masks[e0:e1].astype(np.uint64)
+        assert np.all(np.diff(pg) > 0), "column pages must be ascending and unique"
+        for r in range(128):
+            c = int(codes[r])
+            if c == 15:
+                continue
+            assert r < 16 * n_own
+            slot = int(w[4 + r // 16]) * 16 + r % 16
+            assert slot < own_group.size
+            if row_filter is not None and slot not in row_filter:
+                continue
+            owned[(h, slot)] = owned.get((h, slot), 0) + 1
+            if c == 14:
+                assert own_group[slot] == -1
+                continue
+            assert c < 4 and own_group[slot] >= 0
+            bits = ((mk[:, None] >> (np.uint64(16 * c) + bits16)) & np.uint64(1)).astype(bool)
+            cols = (pg[:, None] * 16 + np.arange(16))[bits]
+            assert np.all(cols < col_slots)
+            for col in cols.tolist():
+                pairs[(h, slot, col)] = pairs.get((h, slot, col), 0) + 1
+    return pairs, owned
+
+
+@pytest.mark.parametrize("name", TINY)
+@pytest.mark.parametrize("which", [0, 1])
+def test_coverage_invariant_tiny(name, which):
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p)
+    pairs, owned = _covered(p, pl, which)
+    assert all(v == 1 for v in pairs.values()), "a pair is computed by two owned rows"
+    own_group = p.q_group if which == 0 else p.kv_group
+    valid_pages = oracle.page_valid_masks(own_group) != 0
+    for h in range(p.heads):
+        M = oracle.token_mask(p.q_group, p.kv_group, _allowed(p, h))
+        if which == 1:
+            M = M.T
+        got = np.zeros_like(M)
+        for (hh, i, j) in pairs:
+            if hh == h:
+                got[i, j] = True
+        assert np.array_equal(got, M)
+        for slot in range(own_group.size):
+            expect = 1 if valid_pages[slot // 16] else 0
+            assert owned.get((h, slot), 0) == expect, (h, slot)
+
+
+@pytest.mark.parametrize("name", ["full", "partial", "vsa", "svg2"])
+def test_page_lists_and_counts_large_sampled(name):
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p)
+    st = pl.stats()
+    assert st["useful_pairs"] == oracle.useful_pairs_closed_form(
+        p.q_group, p.kv_group, p.row_ptr, p.kv_groups, p.n_q_groups, p.n_kv_groups, p.heads)
+    rng = np.random.default_rng(17)
+    n_qb = -(-p.q_slots // 64)
+    for _ in range(12):
+        h = int(rng.integers(p.heads))
+        qb = int(rng.integers(n_qb))
+        A = _allowed(p, h)
+        assert np.array_equal(pl.pages(h, qb), oracle.canonical_pages(p.q_group, p.kv_group, A, qb)), (h, qb)
+    # coverage restricted to a few query rows / key rows of one head
+    h = int(rng.integers(p.heads))
+    A = _allowed(p, h)
+    rows = set(rng.integers(0, p.q_slots, size=6).tolist())
+    pairs, owned = _covered(p, pl, 0, head_filter={h}, row_filter=rows)
+    M = oracle.token_mask(p.q_group, p.kv_group, A, np.array(sorted(rows)))
+    for k, i in enumerate(sorted(rows)):
+        got = sorted(j for (hh, ii, j) in pairs if ii == i)
+        assert got == np.nonzero(M[k])[0].tolist()
+    keys = set(rng.integers(0, p.kv_slots, size=4).tolist())
+    pairs, owned = _covered(p, pl, 1, head_filter={h}, row_filter=keys)
+    Mt = oracle.token_mask(p.q_group, p.kv_group, A)[:, sorted(keys)].T if p.q_slots <= 20000 else None
+    for k, j in enumerate(sorted(keys)):
+        got = sorted(i for (hh, jj, i) in pairs if jj == j)
+        if Mt is not None:
+            exp = np.nonzero(Mt[k])[0].tolist()
+        else:
+            g = p.kv_group[j]
+            exp = [] if g < 0 else np.nonzero((p.q_group >= 0) & A[np.where(p.q_group >= 0, p.q_group, 0), g])[0].tolist()
+        assert got == exp
