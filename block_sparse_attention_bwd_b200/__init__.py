@@ -34,8 +34,9 @@ STATUS_NAMES = {
 }
 
 ENTRY_POINTS = (
-    "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_check", "spattn_plan_stats", "spattn_plan_pages",
-    "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy", "spattn_status_string",
+    "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_check", "spattn_plan_stats", "spattn_profile",
+    "spattn_profile_read", "spattn_plan_pages", "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy",
+    "spattn_status_string",
 )
 
 
@@ -61,7 +62,15 @@ class _Graph(ctypes.Structure):
 class _Stats(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int64) for n in (
         "useful_pairs", "physical_pairs_fwd", "physical_pairs_dkdv", "physical_pairs_dq", "bsa_pairs",
-        "n_work_fwd", "n_work_dkdv", "n_entries_fwd", "n_entries_dkdv", "device_bytes")] + [("plan_ms", ctypes.c_double)]
+        "n_work_fwd", "n_work_dkdv", "n_entries_fwd", "n_entries_dkdv", "device_bytes", "launches_fwd",
+        "launches_bwd")] + [("plan_ms", ctypes.c_double)]
+
+
+class _KernelTimes(ctypes.Structure):
+    _fields_ = [("ms", ctypes.c_double * 5), ("launches", ctypes.c_int64 * 5)]
+
+
+KERNEL_NAMES = ("fwd", "fill", "delta", "dkdv", "dq")
 
 
 _LIB = None
@@ -85,6 +94,8 @@ def _lib():
         lib.spattn_plan_work.argtypes = [P, I32, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64),
                                          ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(ctypes.POINTER(ctypes.c_uint64)),
                                          ctypes.POINTER(I64)]
+        lib.spattn_profile.argtypes = [P, ctypes.c_int]
+        lib.spattn_profile_read.argtypes = [P, ctypes.POINTER(_KernelTimes)]
         lib.spattn_plan_destroy.argtypes = [P]
         lib.spattn_plan_destroy.restype = None
         lib.spattn_status_string.argtypes = [ctypes.c_int]
@@ -151,6 +162,16 @@ class Plan:
         s = _Stats()
         _check(_lib().spattn_plan_stats(self.handle, ctypes.byref(s)), "spattn_plan_stats")
         return {n: getattr(s, n) for n, _ in _Stats._fields_}
+
+    def profile(self, enable: bool):
+        """Start / stop recording per-kernel CUDA events in fwd / bwd calls (clears the record)."""
+        _check(_lib().spattn_profile(self.handle, 1 if enable else 0), "spattn_profile")
+
+    def profile_read(self) -> dict:
+        """{kernel: (summed ms, launches)} of the recorded launches; clears the record."""
+        t = _KernelTimes()
+        _check(_lib().spattn_profile_read(self.handle, ctypes.byref(t)), "spattn_profile_read")
+        return {n: (t.ms[i], t.launches[i]) for i, n in enumerate(KERNEL_NAMES)}
 
     def pages(self, head: int, qblock: int) -> np.ndarray:
         ptr = ctypes.POINTER(ctypes.c_int32)()

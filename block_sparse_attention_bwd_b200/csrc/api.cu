@@ -58,6 +58,25 @@ int check_plan_device(const spattn_plan_s* P) {
   return dev == P->device ? SPATTN_OK : SPATTN_ERR_INVALID_ARG;
 }
 
+// Launch helper: runs `launch` and, while profiling, brackets it with events.
+template <typename F>
+cudaError_t timed(spattn_plan_s* P, int kernel, cudaStream_t s, F&& launch) {
+  if (!P->profiling) return launch();
+  if (P->n_events == P->events.size()) {
+    spattn_plan_s::EventRec r{kernel, nullptr, nullptr};
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return cudaErrorMemoryAllocation;
+    P->events.push_back(r);
+  }
+  auto& r = P->events[P->n_events++];
+  r.kernel = kernel;
+  cudaError_t e = cudaEventRecord(r.start, s);
+  if (e == cudaSuccess) e = launch();
+  if (e == cudaSuccess) e = cudaEventRecord(r.stop, s);
+  return e;
+}
+
+int64_t fill_launches(const std::vector<int32_t>& pages) { return pages.empty() ? 0 : 1; }
+
 TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots) {
   TileArgs a;
   a.work = w.d_work;
@@ -114,10 +133,14 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* O = static_cast<__nv_bfloat16*>(o);
-  cudaError_t e = launch_fwd(D, tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), O, lse, s);
-  if (e == cudaSuccess)
-    e = launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots, O,
-                    nullptr, lse, s);
+  cudaError_t e = timed(plan, SPATTN_K_FWD, s, [&] {
+    return launch_fwd(D, tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), O, lse, s);
+  });
+  if (e == cudaSuccess && !plan->q_invalid_pages.empty())
+    e = timed(plan, SPATTN_K_FILL, s, [&] {
+      return launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots,
+                         O, nullptr, lse, s);
+    });
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }
 
@@ -139,20 +162,30 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
   auto* dQ = static_cast<__nv_bfloat16*>(dq);
   auto* dK = static_cast<__nv_bfloat16*>(dk);
   auto* dV = static_cast<__nv_bfloat16*>(dv);
-  cudaError_t e = launch_delta(D, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o),
-                               plan->d_delta, bh * plan->q.slots, s);
+  cudaError_t e = timed(plan, SPATTN_K_DELTA, s, [&] {
+    return launch_delta(D, static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(d_o), plan->d_delta,
+                        bh * plan->q.slots, s);
+  });
   if (e == cudaSuccess)
-    e = launch_dkdv(D, tk, tv, tq, tdo, tile_args(plan, plan->wk, plan->k.slots, plan->q.slots), lse, plan->d_delta,
-                    dK, dV, s);
+    e = timed(plan, SPATTN_K_DKDV, s, [&] {
+      return launch_dkdv(D, tk, tv, tq, tdo, tile_args(plan, plan->wk, plan->k.slots, plan->q.slots), lse,
+                         plan->d_delta, dK, dV, s);
+    });
   if (e == cudaSuccess)
-    e = launch_dq(D, tq, tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, plan->d_delta,
-                  dQ, s);
-  if (e == cudaSuccess)
-    e = launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots, dK,
-                    dV, nullptr, s);
-  if (e == cudaSuccess)
-    e = launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots, dQ,
-                    nullptr, nullptr, s);
+    e = timed(plan, SPATTN_K_DQ, s, [&] {
+      return launch_dq(D, tq, tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse,
+                       plan->d_delta, dQ, s);
+    });
+  if (e == cudaSuccess && !plan->k_invalid_pages.empty())
+    e = timed(plan, SPATTN_K_FILL, s, [&] {
+      return launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots,
+                         dK, dV, nullptr, s);
+    });
+  if (e == cudaSuccess && !plan->q_invalid_pages.empty())
+    e = timed(plan, SPATTN_K_FILL, s, [&] {
+      return launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots,
+                         dQ, nullptr, nullptr, s);
+    });
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }
 
@@ -181,8 +214,36 @@ int spattn_plan_stats(spattn_plan_t plan, spattn_stats* s) {
   s->n_entries_fwd = static_cast<int64_t>(plan->wq.pages.size());
   s->n_entries_dkdv = static_cast<int64_t>(plan->wk.pages.size());
   s->device_bytes = plan->device_bytes;
+  s->launches_fwd = (plan->wq.n_work > 0) + fill_launches(plan->q_invalid_pages);
+  s->launches_bwd = 1 + (plan->wk.n_work > 0) + (plan->wq.n_work > 0) + fill_launches(plan->k_invalid_pages) +
+                    fill_launches(plan->q_invalid_pages);
   s->plan_ms = plan->plan_ms;
   return SPATTN_OK;
+}
+
+int spattn_profile(spattn_plan_t plan, int enable) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  plan->profiling = enable != 0;
+  plan->n_events = 0;
+  return SPATTN_OK;
+}
+
+int spattn_profile_read(spattn_plan_t plan, spattn_kernel_times* out) {
+  if (!plan || !out) return SPATTN_ERR_INVALID_ARG;
+  std::memset(out, 0, sizeof(*out));
+  int st = SPATTN_OK;
+  for (size_t i = 0; i < plan->n_events; ++i) {
+    auto& r = plan->events[i];
+    float ms = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&ms, r.start, r.stop) != cudaSuccess) {
+      st = SPATTN_ERR_CUDA;
+      continue;
+    }
+    out->ms[r.kernel] += ms;
+    out->launches[r.kernel] += 1;
+  }
+  plan->n_events = 0;
+  return st;
 }
 
 int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const int32_t** pages, int64_t* n) {

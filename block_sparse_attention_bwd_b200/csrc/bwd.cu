@@ -61,15 +61,23 @@ __global__ void delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfl
 }
 
 // ----------------------------------------------------------------------------
-// K3: dK, dV (key-owned tiles, query pages as columns)
+// K3: dK, dV (key-owned tiles, query pages as columns, 64 columns per step)
 // ----------------------------------------------------------------------------
+// TMEM columns: S^T / P^T double buffer at 0 and 64, dP^T / dS^T double
+// buffer at 128 and 192, dV at 256, dK at 256 + D.  The MMAs of step c+1
+// (S^T, dP^T) run while the row threads turn step c into P^T and dS^T.
+constexpr int kBwdStepPages = 4;                  // 64 columns per step
+constexpr int kStageChunk = 64 * 128;             // one 64-column chunk of a 64-row stage
+
 template <int D>
 struct DkvCfg {
   static constexpr int kNch = D / 64;
-  static constexpr int kTile = kNch * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kStage = 2 * kTile + 2 * 128 * 4;  // Q, dO tiles + LSE2, Delta of 128 columns
-  static constexpr int kSmem = 2 * kTile + kStages * kStage + 1024 + 256;
+  static constexpr int kTile = kNch * kChunkBytes;     // owned 128-row tile
+  static constexpr int kStageTile = kNch * kStageChunk;  // 64-row column stage
+  static constexpr int kQStages = (D == 128) ? 4 : 6;
+  static constexpr int kDStages = (D == 128) ? 4 : 6;
+  static constexpr int kLdBytes = 2 * 64 * 4;          // LSE2 and Delta of 64 columns
+  static constexpr int kSmem = 2 * kTile + kQStages * kStageTile + kDStages * (kStageTile + kLdBytes) + 1024 + 512;
 };
 
 template <int D>
@@ -82,42 +90,52 @@ __global__ void __launch_bounds__(256, 1)
                 __nv_bfloat16* __restrict__ out_dv, int64_t kv_slots, int64_t q_slots, float sl2, float scale,
                 int* err) {
   using C = DkvCfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int QS = C::kQStages, DS = C::kDStages, NP = kBwdStepPages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;
   uint8_t* sV = smem + C::kTile;
-  uint8_t* sStage = smem + 2 * C::kTile;  // stage s: Q, dO, LSE2[128], Delta[128]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sStage + NS * C::kStage);
+  uint8_t* sQ = smem + 2 * C::kTile;                 // Q stage s at sQ + s*kStageTile
+  uint8_t* sDO = sQ + QS * C::kStageTile;            // dO stage s at sDO + s*kStageTile
+  float* sLD = reinterpret_cast<float*>(sDO + DS * C::kStageTile);  // stage s: LSE2[64], Delta[64]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLD) + DS * C::kLdBytes);
   uint64_t* own_full = bars;
-  uint64_t* q_full = bars + 1;
-  uint64_t* do_full = q_full + NS;
-  uint64_t* ld_full = do_full + NS;
-  uint64_t* stage_empty = ld_full + NS;
-  uint64_t* st_full = stage_empty + NS;
-  uint64_t* pt_full = st_full + 1;
-  uint64_t* acc_done = pt_full + 1;
-  uint64_t* drain = acc_done + 1;
+  uint64_t* q_full = own_full + 1;
+  uint64_t* q_empty = q_full + QS;
+  uint64_t* do_full = q_empty + QS;
+  uint64_t* do_empty = do_full + DS;
+  uint64_t* ld_full = do_empty + DS;
+  uint64_t* st_full = ld_full + DS;  // [2]
+  uint64_t* pt_full = st_full + 2;   // [2]
+  uint64_t* acc_done = pt_full + 2;
+  uint64_t* acc_step = acc_done + 1;  // completes once per step's dV, dK MMAs
+  uint64_t* drain = acc_step + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
 
   const Work wk = load_work(work, blockIdx.x);
   const int n_cols = wk.e1 - wk.e0;
-  const int n_steps = (n_cols + kStepPages - 1) / kStepPages;
+  const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(own_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    mbar_init(acc_step, 1);
+    for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
-      mbar_init(&do_full[s], 1);
-      mbar_init(&ld_full[s], 32);
-      mbar_init(&stage_empty[s], 1);
+      mbar_init(&q_empty[s], 1);
     }
-    mbar_init(st_full, 1);
-    mbar_init(pt_full, 128);
+    for (int s = 0; s < DS; ++s) {
+      mbar_init(&do_full[s], 1);
+      mbar_init(&do_empty[s], 1);
+      mbar_init(&ld_full[s], 32);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&st_full[b], 1);
+      mbar_init(&pt_full[b], 128);
+    }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
@@ -127,15 +145,10 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tST = tmem, tDPT = tmem + 128, tDV = tmem + 256, tDK = tmem + 256 + D;
-
-  auto stage_q = [&](int s) { return sStage + s * C::kStage; };
-  auto stage_do = [&](int s) { return sStage + s * C::kStage + C::kTile; };
-  auto stage_l = [&](int s) { return reinterpret_cast<float*>(sStage + s * C::kStage + 2 * C::kTile); };
-  auto stage_d = [&](int s) { return reinterpret_cast<float*>(sStage + s * C::kStage + 2 * C::kTile) + 128; };
+  const uint32_t tDV = tmem + 256, tDK = tmem + 256 + D;
 
   if (warp == 0) {
-    // ---------------- producer (lane 0: TMA; all lanes: LSE / Delta) ----------------
+    // ---------------- producer (lane 0: TMA; all lanes: LSE2 / Delta) ----------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -148,47 +161,48 @@ __global__ void __launch_bounds__(256, 1)
           tma_load_3d(sV + c * kChunkBytes + p * 2048, &tm_v, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
         }
     }
-    int issued = 0;
+    int q_issued = 0, d_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
-      const int s = st % NS;
-      if (st >= NS) {
-        bool ok = mbar_wait(&stage_empty[s], ((st / NS) - 1) & 1, ab);
+      const int qs = st % QS, ds = st % DS;
+      const int n = min(NP, n_cols - st * NP);
+      const int32_t* pg = col_pages + wk.e0 + st * NP;
+      if (st >= QS) {
+        const bool ok = mbar_wait(&q_empty[qs], ((st / QS) - 1) & 1, ab);
         if (!__all_sync(0xffffffffu, ok)) break;
       }
-      const int n = min(kStepPages, n_cols - st * kStepPages);
-      const int32_t* pg = col_pages + wk.e0 + st * kStepPages;
       if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j)
-          for (int c = 0; c < C::kNch; ++c)
-            tma_load_3d(stage_q(s) + c * kChunkBytes + j * 2048, &tm_q, c * 64, __ldg(pg + j) * 16, wk.bh, &q_full[s]);
-        mbar_arrive_expect_tx(&do_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j)
-          for (int c = 0; c < C::kNch; ++c)
-            tma_load_3d(stage_do(s) + c * kChunkBytes + j * 2048, &tm_do, c * 64, __ldg(pg + j) * 16, wk.bh,
-                        &do_full[s]);
+        mbar_arrive_expect_tx(&q_full[qs], n * C::kNch * 2048);
+        load_pages<C::kNch>(sQ + qs * C::kStageTile, kStageChunk, &tm_q, pg, n, wk.bh, &q_full[qs]);
       }
-      float* sl = stage_l(s);
-      float* sd = stage_d(s);
-      for (int idx = lane; idx < 16 * n; idx += 32) {
-        const int64_t slot = static_cast<int64_t>(__ldg(pg + (idx >> 4))) * 16 + (idx & 15);
+      q_issued = st + 1;
+      if (st >= DS) {
+        const bool ok = mbar_wait(&do_empty[ds], ((st / DS) - 1) & 1, ab);
+        if (!__all_sync(0xffffffffu, ok)) break;
+      }
+      if (lane == 0) {
+        mbar_arrive_expect_tx(&do_full[ds], n * C::kNch * 2048);
+        load_pages<C::kNch>(sDO + ds * C::kStageTile, kStageChunk, &tm_do, pg, n, wk.bh, &do_full[ds]);
+      }
+      d_issued = st + 1;
+      float* sl = sLD + ds * 128;
+      for (int idx = lane; idx < 16 * NP; idx += 32) {
         float l2 = 0.f, dl = 0.f;
-        if (slot < q_slots) {
-          const int64_t off = static_cast<int64_t>(wk.bh) * q_slots + slot;
-          l2 = __ldg(lse + off) * kLog2e;
-          dl = __ldg(delta + off);
+        if (idx < 16 * n) {
+          const int64_t slot = static_cast<int64_t>(__ldg(pg + (idx >> 4))) * 16 + (idx & 15);
+          if (slot < q_slots) {
+            const int64_t off = static_cast<int64_t>(wk.bh) * q_slots + slot;
+            l2 = __ldg(lse + off) * kLog2e;
+            dl = __ldg(delta + off);
+          }
         }
         sl[idx] = l2;
-        sd[idx] = dl;
+        sl[64 + idx] = dl;
       }
-      mbar_arrive(&ld_full[s]);
-      issued = st + 1;
+      mbar_arrive(&ld_full[ds]);
     }
     if (lane == 0) {
-      for (int st = max(0, issued - NS); st < issued; ++st) {
-        mbar_wait_drain(&q_full[st % NS], (st / NS) & 1);
-        mbar_wait_drain(&do_full[st % NS], (st / NS) & 1);
-      }
+      for (int st = max(0, q_issued - QS); st < q_issued; ++st) mbar_wait_drain(&q_full[st % QS], (st / QS) & 1);
+      for (int st = max(0, d_issued - DS); st < d_issued; ++st) mbar_wait_drain(&do_full[st % DS], (st / DS) & 1);
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
@@ -198,37 +212,48 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
       bool ok = mbar_wait(own_full, 0, ab);
       tc_fence_after();
+      auto issue_acc = [&](int st) -> bool {
+        const int b = st & 1, qs = st % QS, ds = st % DS;
+        if (!mbar_wait(&pt_full[b], (st >> 1) & 1, ab)) return false;
+        tc_fence_after();
+        const int n = min(NP, n_cols - st * NP);
+        const uint32_t q_addr = smem_u32(sQ + qs * C::kStageTile), do_addr = smem_u32(sDO + ds * C::kStageTile);
+        for (int j = 0; j < n; ++j)
+          umma_ts(tDV, tmem + 64 * b + 8 * j, sdesc_sw128(do_addr + j * 2048, kStageChunk, 1024), idesc_acc,
+                  (st > 0 || j > 0) ? 1u : 0u);
+        umma_commit(&do_empty[ds]);
+        for (int j = 0; j < n; ++j)
+          umma_ts(tDK, tmem + 128 + 64 * b + 8 * j, sdesc_sw128(q_addr + j * 2048, kStageChunk, 1024), idesc_acc,
+                  (st > 0 || j > 0) ? 1u : 0u);
+        umma_commit(&q_empty[qs]);
+        umma_commit(acc_step);
+        return true;
+      };
       for (int st = 0; ok && st < n_steps; ++st) {
-        const int s = st % NS;
-        const int n = min(kStepPages, n_cols - st * kStepPages);
+        const int b = st & 1, qs = st % QS, ds = st % DS;
+        const int n = min(NP, n_cols - st * NP);
         const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t q_addr = smem_u32(stage_q(s)), do_addr = smem_u32(stage_do(s));
-        if (!mbar_wait(&q_full[s], (st / NS) & 1, ab)) { ok = false; break; }
+        const uint32_t q_addr = smem_u32(sQ + qs * C::kStageTile), do_addr = smem_u32(sDO + ds * C::kStageTile);
+        // buffers b still feed dV(st-2) / dK(st-2) as TMEM A operands
+        if (st >= 2 && !mbar_wait(acc_step, (st - 2) & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(&q_full[qs], (st / QS) & 1, ab)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(tST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s, kk > 0);
+          umma_ss(tmem + 64 * b, sdesc_sw128(k_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(q_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
         }
-        if (!mbar_wait(&do_full[s], (st / NS) & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(&do_full[ds], (st / DS) & 1, ab)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(tDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), idesc_s, kk > 0);
+          umma_ss(tmem + 128 + 64 * b, sdesc_sw128(v_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(do_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
         }
-        umma_commit(st_full);
-        if (!mbar_wait(pt_full, st & 1, ab)) { ok = false; break; }
-        tc_fence_after();
-        for (int j = 0; j < n; ++j)
-          umma_ts(tDV, tST + 8 * j, sdesc_sw128(do_addr + j * 2048, kChunkBytes, 1024), idesc_acc,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        for (int j = 0; j < n; ++j)
-          umma_ts(tDK, tDPT + 8 * j, sdesc_sw128(q_addr + j * 2048, kChunkBytes, 1024), idesc_acc,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&stage_empty[s]);
+        umma_commit(&st_full[b]);
+        if (st >= 1 && !issue_acc(st - 1)) ok = false;
       }
-      if (ok && n_steps > 0) umma_commit(acc_done);
+      if (ok && n_steps > 0 && issue_acc(n_steps - 1)) umma_commit(acc_done);
       umma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
@@ -240,47 +265,59 @@ __global__ void __launch_bounds__(256, 1)
     const uint32_t code = wk.row_code(row);
     const int seg = code < 4 ? static_cast<int>(code) : -1;
     bool ok = true;
+    uint32_t mw[2];
+    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
-      const int s = st % NS;
-      const int n = min(kStepPages, n_cols - st * kStepPages);
-      const int N = 16 * n;
-      uint32_t mw[4];
-      step_masks(col_masks, wk.e0 + st * kStepPages, n, seg, mw);
-      ok = mbar_wait(st_full, st & 1, ab) && mbar_wait(&ld_full[s], (st / NS) & 1, ab);
+      const int b = st & 1, ds = st % DS;
+      const int N = 16 * min(NP, n_cols - st * NP);
+      ok = mbar_wait(&st_full[b], (st >> 1) & 1, ab) && mbar_wait(&ld_full[ds], (st / DS) & 1, ab);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const float* sl = stage_l(s);
-      const float* sd = stage_d(s);
+      uint32_t a[2][32], d[2][32];
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
+      for (int pc = 0; pc < 2; ++pc)
         if (pc * 32 < N) {
-          uint32_t a[32], b[32];
-          tmem_ld32(tST + lane_off + pc * 32, a);
-          tmem_ld32(tDPT + lane_off + pc * 32, b);
-          tmem_wait_ld();
+          tmem_ld32(tmem + 64 * b + lane_off + pc * 32, a[pc]);
+          tmem_ld32(tmem + 128 + 64 * b + lane_off + pc * 32, d[pc]);
+        }
+      uint32_t mw_next[2] = {0u, 0u};
+      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
+      tmem_wait_ld();
+      const float4* sl4 = reinterpret_cast<const float4*>(sLD + ds * 128);
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        if (pc * 32 < N) {
           uint32_t pp[16], pd[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float pv[2], dv[2];
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 L = sl4[pc * 8 + i4];
+            const float4 Dl = sl4[16 + pc * 8 + i4];
+            const float lv[4] = {L.x, L.y, L.z, L.w};
+            const float dv[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
+            float pv[4], sv[4];
 #pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int c = pc * 32 + 2 * i + h;
-              const bool on = (mw[pc] >> (2 * i + h)) & 1u;
-              const float p = on ? ex2(__uint_as_float(a[2 * i + h]) * sl2 - sl[c]) : 0.f;
+            for (int h = 0; h < 4; ++h) {
+              const int i = 4 * i4 + h;
+              const bool on = (mw[pc] >> i) & 1u;
+              const float p = on ? ex2(fmaf(__uint_as_float(a[pc][i]), sl2, -lv[h])) : 0.f;
               pv[h] = p;
-              dv[h] = on ? p * (__uint_as_float(b[2 * i + h]) - sd[c]) : 0.f;
+              sv[h] = on ? p * (__uint_as_float(d[pc][i]) - dv[h]) : 0.f;
             }
-            pp[i] = pack_bf16(pv[0], pv[1]);
-            pd[i] = pack_bf16(dv[0], dv[1]);
+            pp[2 * i4] = pack_bf16(pv[0], pv[1]);
+            pp[2 * i4 + 1] = pack_bf16(pv[2], pv[3]);
+            pd[2 * i4] = pack_bf16(sv[0], sv[1]);
+            pd[2 * i4 + 1] = pack_bf16(sv[2], sv[3]);
           }
-          tmem_st16(tST + lane_off + pc * 16, pp);
-          tmem_st16(tDPT + lane_off + pc * 16, pd);
+          tmem_st16(tmem + 64 * b + lane_off + pc * 16, pp);
+          tmem_st16(tmem + 128 + 64 * b + lane_off + pc * 16, pd);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(pt_full);
+      mbar_arrive(&pt_full[b]);
+      mw[0] = mw_next[0];
+      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, ab));
@@ -323,12 +360,16 @@ __global__ void __launch_bounds__(256, 1)
 // ----------------------------------------------------------------------------
 // K4: dQ (query-owned tiles, key pages as columns; the forward lists)
 // ----------------------------------------------------------------------------
+// TMEM columns: S / dS double buffer at 0 and 64, dP double buffer at 128
+// and 192, dQ at 256.  K stays in its stage until the dQ MMA of its step.
 template <int D>
 struct DqCfg {
   static constexpr int kNch = D / 64;
   static constexpr int kTile = kNch * kChunkBytes;
-  static constexpr int kStages = (D == 128) ? 2 : 4;
-  static constexpr int kSmem = 2 * kTile + kStages * 2 * kTile + 1024 + 256;
+  static constexpr int kStageTile = kNch * kStageChunk;
+  static constexpr int kKStages = (D == 128) ? 5 : 8;
+  static constexpr int kVStages = (D == 128) ? 4 : 8;
+  static constexpr int kSmem = 2 * kTile + (kKStages + kVStages) * kStageTile + 1024 + 512;
 };
 
 template <int D>
@@ -339,41 +380,50 @@ __global__ void __launch_bounds__(256, 1)
               const uint64_t* __restrict__ col_masks, const float* __restrict__ lse, const float* __restrict__ delta,
               __nv_bfloat16* __restrict__ out_dq, int64_t q_slots, float sl2, float scale, int* err) {
   using C = DqCfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int KS = C::kKStages, VS = C::kVStages, NP = kBwdStepPages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;
   uint8_t* sDO = smem + C::kTile;
-  uint8_t* sKV = smem + 2 * C::kTile;  // stage s: K at sKV + 2*s*kTile, V right after
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sKV + NS * 2 * C::kTile);
+  uint8_t* sK = smem + 2 * C::kTile;       // K stage s at sK + s*kStageTile
+  uint8_t* sV = sK + KS * C::kStageTile;   // V stage s at sV + s*kStageTile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kStageTile);
   uint64_t* own_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + NS;
-  uint64_t* kv_empty = v_full + NS;
-  uint64_t* sd_full = kv_empty + NS;
-  uint64_t* ds_full = sd_full + 1;
-  uint64_t* acc_done = ds_full + 1;
-  uint64_t* drain = acc_done + 1;
+  uint64_t* k_full = own_full + 1;
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* sd_full = v_empty + VS;  // [2]
+  uint64_t* ds_full = sd_full + 2;   // [2]
+  uint64_t* acc_done = ds_full + 2;
+  uint64_t* dq_step = acc_done + 1;  // completes once per step's dQ MMAs
+  uint64_t* drain = dq_step + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
 
   const Work wk = load_work(work, blockIdx.x);
   const int n_cols = wk.e1 - wk.e0;
-  const int n_steps = (n_cols + kStepPages - 1) / kStepPages;
+  const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(own_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
     }
-    mbar_init(sd_full, 1);
-    mbar_init(ds_full, 128);
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sd_full[b], 1);
+      mbar_init(&ds_full[b], 128);
+    }
     mbar_init(acc_done, 1);
+    mbar_init(dq_step, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
   }
@@ -382,7 +432,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tS = tmem, tDP = tmem + 128, tDQ = tmem + 256;
+  const uint32_t tDQ = tmem + 256;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -396,28 +446,22 @@ __global__ void __launch_bounds__(256, 1)
           tma_load_3d(sQ + c * kChunkBytes + p * 2048, &tm_q, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
           tma_load_3d(sDO + c * kChunkBytes + p * 2048, &tm_do, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
         }
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int st = 0; st < n_steps; ++st) {
-        const int s = st % NS;
-        if (st >= NS && !mbar_wait(&kv_empty[s], ((st / NS) - 1) & 1, ab)) break;
-        const int n = min(kStepPages, n_cols - st * kStepPages);
-        uint8_t* kd = sKV + 2 * s * C::kTile;
-        uint8_t* vd = kd + C::kTile;
-        const int32_t* pg = col_pages + wk.e0 + st * kStepPages;
-        mbar_arrive_expect_tx(&k_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j)
-          for (int c = 0; c < C::kNch; ++c)
-            tma_load_3d(kd + c * kChunkBytes + j * 2048, &tm_k, c * 64, __ldg(pg + j) * 16, wk.bh, &k_full[s]);
-        mbar_arrive_expect_tx(&v_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j)
-          for (int c = 0; c < C::kNch; ++c)
-            tma_load_3d(vd + c * kChunkBytes + j * 2048, &tm_v, c * 64, __ldg(pg + j) * 16, wk.bh, &v_full[s]);
-        issued = st + 1;
+        const int ks = st % KS, vs = st % VS;
+        const int n = min(NP, n_cols - st * NP);
+        const int32_t* pg = col_pages + wk.e0 + st * NP;
+        if (st >= KS && !mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+        load_pages<C::kNch>(sK + ks * C::kStageTile, kStageChunk, &tm_k, pg, n, wk.bh, &k_full[ks]);
+        k_issued = st + 1;
+        if (st >= VS && !mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
+        load_pages<C::kNch>(sV + vs * C::kStageTile, kStageChunk, &tm_v, pg, n, wk.bh, &v_full[vs]);
+        v_issued = st + 1;
       }
-      for (int st = max(0, issued - NS); st < issued; ++st) {
-        mbar_wait_drain(&k_full[st % NS], (st / NS) & 1);
-        mbar_wait_drain(&v_full[st % NS], (st / NS) & 1);
-      }
+      for (int st = max(0, k_issued - KS); st < k_issued; ++st) mbar_wait_drain(&k_full[st % KS], (st / KS) & 1);
+      for (int st = max(0, v_issued - VS); st < v_issued; ++st) mbar_wait_drain(&v_full[st % VS], (st / VS) & 1);
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
@@ -426,35 +470,43 @@ __global__ void __launch_bounds__(256, 1)
       const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
       bool ok = mbar_wait(own_full, 0, ab);
       tc_fence_after();
-      for (int st = 0; ok && st < n_steps; ++st) {
-        const int s = st % NS;
-        const int n = min(kStepPages, n_cols - st * kStepPages);
-        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t k_addr = smem_u32(sKV + 2 * s * C::kTile);
-        const uint32_t v_addr = k_addr + C::kTile;
-        if (!mbar_wait(&k_full[s], (st / NS) & 1, ab)) { ok = false; break; }
+      auto issue_dq = [&](int st) -> bool {
+        const int b = st & 1, ks = st % KS;
+        if (!mbar_wait(&ds_full[b], (st >> 1) & 1, ab)) return false;
         tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(tS, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0);
-        }
-        if (!mbar_wait(&v_full[s], (st / NS) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(tDP, sdesc_sw128(do_addr + off, 16, 1024), sdesc_sw128(v_addr + off, 16, 1024), idesc_s, kk > 0);
-        }
-        umma_commit(sd_full);
-        if (!mbar_wait(ds_full, st & 1, ab)) { ok = false; break; }
-        tc_fence_after();
+        const int n = min(NP, n_cols - st * NP);
+        const uint32_t k_addr = smem_u32(sK + ks * C::kStageTile);
         for (int j = 0; j < n; ++j)
-          umma_ts(tDQ, tS + 8 * j, sdesc_sw128(k_addr + j * 2048, kChunkBytes, 1024), idesc_acc,
+          umma_ts(tDQ, tmem + 64 * b + 8 * j, sdesc_sw128(k_addr + j * 2048, kStageChunk, 1024), idesc_acc,
                   (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&kv_empty[s]);
+        umma_commit(&k_empty[ks]);
+        umma_commit(dq_step);
+        return true;
+      };
+      for (int st = 0; ok && st < n_steps; ++st) {
+        const int b = st & 1, ks = st % KS, vs = st % VS;
+        const int n = min(NP, n_cols - st * NP);
+        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+        const uint32_t k_addr = smem_u32(sK + ks * C::kStageTile), v_addr = smem_u32(sV + vs * C::kStageTile);
+        // buffer b still feeds dQ(st-2) as its TMEM A operand
+        if (st >= 2 && !mbar_wait(dq_step, (st - 2) & 1, ab)) { ok = false; break; }
+        if (!mbar_wait(&k_full[ks], (st / KS) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + 64 * b, sdesc_sw128(q_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(k_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
+        if (!mbar_wait(&v_full[vs], (st / VS) & 1, ab)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss(tmem + 128 + 64 * b, sdesc_sw128(do_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(v_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
+        umma_commit(&v_empty[vs]);
+        umma_commit(&sd_full[b]);
+        if (st >= 1 && !issue_dq(st - 1)) ok = false;
       }
-      if (ok && n_steps > 0) umma_commit(acc_done);
+      if (ok && n_steps > 0 && issue_dq(n_steps - 1)) umma_commit(acc_done);
       umma_commit(drain);
       mbar_wait_drain(drain, 0);
     }
@@ -471,39 +523,47 @@ __global__ void __launch_bounds__(256, 1)
     const float lse2 = (valid_slot && seg >= 0) ? __ldg(lse + roff) * kLog2e : 0.f;
     const float dl = (valid_slot && seg >= 0) ? __ldg(delta + roff) : 0.f;
     bool ok = true;
+    uint32_t mw[2];
+    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
-      const int n = min(kStepPages, n_cols - st * kStepPages);
-      const int N = 16 * n;
-      uint32_t mw[4];
-      step_masks(col_masks, wk.e0 + st * kStepPages, n, seg, mw);
-      ok = __all_sync(0xffffffffu, mbar_wait(sd_full, st & 1, ab));
+      const int b = st & 1;
+      const int N = 16 * min(NP, n_cols - st * NP);
+      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
+      uint32_t a[2][32], d[2][32];
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
+      for (int pc = 0; pc < 2; ++pc)
         if (pc * 32 < N) {
-          uint32_t a[32], b[32];
-          tmem_ld32(tS + lane_off + pc * 32, a);
-          tmem_ld32(tDP + lane_off + pc * 32, b);
-          tmem_wait_ld();
+          tmem_ld32(tmem + 64 * b + lane_off + pc * 32, a[pc]);
+          tmem_ld32(tmem + 128 + 64 * b + lane_off + pc * 32, d[pc]);
+        }
+      uint32_t mw_next[2] = {0u, 0u};
+      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
+      tmem_wait_ld();
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        if (pc * 32 < N) {
           uint32_t pd[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            float dv[2];
+            float sv[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const bool on = (mw[pc] >> (2 * i + h)) & 1u;
-              const float p = on ? ex2(__uint_as_float(a[2 * i + h]) * sl2 - lse2) : 0.f;
-              dv[h] = on ? p * (__uint_as_float(b[2 * i + h]) - dl) : 0.f;
+              const float p = on ? ex2(fmaf(__uint_as_float(a[pc][2 * i + h]), sl2, -lse2)) : 0.f;
+              sv[h] = on ? p * (__uint_as_float(d[pc][2 * i + h]) - dl) : 0.f;
             }
-            pd[i] = pack_bf16(dv[0], dv[1]);
+            pd[i] = pack_bf16(sv[0], sv[1]);
           }
-          tmem_st16(tS + lane_off + pc * 16, pd);
+          tmem_st16(tmem + 64 * b + lane_off + pc * 16, pd);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(ds_full);
+      mbar_arrive(&ds_full[b]);
+      mw[0] = mw_next[0];
+      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, ab));

@@ -28,10 +28,11 @@ using namespace dev;
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kNch = D / 64;                      // 64-column chunks
-  static constexpr int kTile = kNch * kChunkBytes;         // one 128-row operand
-  static constexpr int kStages = (D == 128) ? 2 : 4;       // K/V ring depth
-  static constexpr int kSmem = kTile * (1 + 2 * kStages) + 1024 + 256;
+  static constexpr int kNch = D / 64;                  // 64-column chunks
+  static constexpr int kTile = kNch * kChunkBytes;     // one 128-row operand
+  static constexpr int kKStages = (D == 128) ? 3 : 6;  // K ring depth
+  static constexpr int kVStages = (D == 128) ? 3 : 6;  // V ring depth
+  static constexpr int kSmem = kTile * (1 + kKStages + kVStages) + 1024 + 512;
 };
 
 // Rescale O only when the running max grows by more than 2^8 (log2 units):
@@ -46,18 +47,20 @@ __global__ void __launch_bounds__(256, 1)
                __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
                int* err) {
   using C = FwdCfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int KS = C::kKStages, VS = C::kVStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sKV = smem + C::kTile;  // stage s: K at sKV + 2*s*kTile, V right after
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kTile * (1 + 2 * NS));
+  uint8_t* sK = smem + C::kTile;          // K stage s at sK + s*kTile
+  uint8_t* sV = sK + KS * C::kTile;       // V stage s at sV + s*kTile
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kTile);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + NS;
-  uint64_t* kv_empty = v_full + NS;
-  uint64_t* s_full = kv_empty + NS;  // [2]
-  uint64_t* p_full = s_full + 2;     // [2]
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + KS;
+  uint64_t* v_full = k_empty + KS;
+  uint64_t* v_empty = v_full + VS;
+  uint64_t* s_full = v_empty + VS;  // [2]
+  uint64_t* p_full = s_full + 2;    // [2]
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 1;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
@@ -72,10 +75,13 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(q_full, 1);
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -90,11 +96,11 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tO = tmem + 256;
+  const uint32_t tO = tmem + 256;  // S buffers at columns 0 and 128
 
   if (warp == 0) {
     if (lane == 0) {
-      // ---------------- producer ----------------
+      // ---------------- producer: K runs ahead of V ----------------
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -102,31 +108,23 @@ __global__ void __launch_bounds__(256, 1)
       for (int p = 0; p < wk.n_own; ++p)
         for (int c = 0; c < C::kNch; ++c)
           tma_load_3d(sQ + c * kChunkBytes + p * 2048, &tm_q, c * 64, wk.own_page(p) * 16, wk.bh, q_full);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int st = 0; st < n_steps; ++st) {
-        const int s = st % NS;
-        if (st >= NS && !mbar_wait(&kv_empty[s], ((st / NS) - 1) & 1, ab)) break;
         const int n = min(kStepPages, n_cols - st * kStepPages);
-        uint8_t* kd = sKV + 2 * s * C::kTile;
-        uint8_t* vd = kd + C::kTile;
         const int32_t* pg = col_pages + wk.e0 + st * kStepPages;
-        mbar_arrive_expect_tx(&k_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j) {
-          const int row = __ldg(pg + j) * 16;
-          for (int c = 0; c < C::kNch; ++c) tma_load_3d(kd + c * kChunkBytes + j * 2048, &tm_k, c * 64, row, wk.bh, &k_full[s]);
-        }
-        mbar_arrive_expect_tx(&v_full[s], n * C::kNch * 2048);
-        for (int j = 0; j < n; ++j) {
-          const int row = __ldg(pg + j) * 16;
-          for (int c = 0; c < C::kNch; ++c) tma_load_3d(vd + c * kChunkBytes + j * 2048, &tm_v, c * 64, row, wk.bh, &v_full[s]);
-        }
-        issued = st + 1;
+        const int ks = st % KS, vs = st % VS;
+        if (st >= KS && !mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+        load_pages<C::kNch>(sK + ks * C::kTile, kChunkBytes, &tm_k, pg, n, wk.bh, &k_full[ks]);
+        k_issued = st + 1;
+        if (st >= VS && !mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab)) break;
+        mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
+        load_pages<C::kNch>(sV + vs * C::kTile, kChunkBytes, &tm_v, pg, n, wk.bh, &v_full[vs]);
+        v_issued = st + 1;
       }
-      // make sure no copy is still landing in shared memory when the CTA exits
-      for (int st = max(0, issued - NS); st < issued; ++st) {
-        mbar_wait_drain(&k_full[st % NS], (st / NS) & 1);
-        mbar_wait_drain(&v_full[st % NS], (st / NS) & 1);
-      }
+      // no copy may still be landing in shared memory when the CTA exits
+      for (int st = max(0, k_issued - KS); st < k_issued; ++st) mbar_wait_drain(&k_full[st % KS], (st / KS) & 1);
+      for (int st = max(0, v_issued - VS); st < v_issued; ++st) mbar_wait_drain(&v_full[st % VS], (st / VS) & 1);
       mbar_wait_drain(q_full, 0);
     }
   } else if (warp == 1) {
@@ -137,29 +135,36 @@ __global__ void __launch_bounds__(256, 1)
       bool ok = mbar_wait(q_full, 0, ab);
       tc_fence_after();
       auto issue_pv = [&](int st) -> bool {
-        const int b = st & 1, s = st % NS;
+        const int b = st & 1, vs = st % VS;
         if (!mbar_wait(&p_full[b], (st >> 1) & 1, ab)) return false;
-        if (!mbar_wait(&v_full[s], (st / NS) & 1, ab)) return false;
+        if (!mbar_wait(&v_full[vs], (st / VS) & 1, ab)) return false;
         tc_fence_after();
         const int n = min(kStepPages, n_cols - st * kStepPages);
-        const uint32_t v_addr = smem_u32(sKV + 2 * s * C::kTile + C::kTile);
+        const uint32_t v_addr = smem_u32(sV + vs * C::kTile);
         for (int j = 0; j < n; ++j)
           umma_ts(tO, tmem + 128 * b + 8 * j, sdesc_sw128(v_addr + j * 2048, kChunkBytes, 1024), idesc_pv,
                   (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&kv_empty[s]);
+        umma_commit(&v_empty[vs]);
         umma_commit(o_done);
         return true;
       };
       for (int st = 0; ok && st < n_steps; ++st) {
-        const int s = st % NS, b = st & 1;
-        if (!mbar_wait(&k_full[s], (st / NS) & 1, ab)) {
+        const int ks = st % KS, b = st & 1;
+        if (!mbar_wait(&k_full[ks], (st / KS) & 1, ab)) {
+          ok = false;
+          break;
+        }
+        // buffer b still holds P(st-2), the TMEM A operand of PV(st-2); let
+        // that MMA finish before S(st) overwrites it (waited every step, in
+        // order, so the parity is unambiguous)
+        if (st >= 2 && !mbar_wait(o_done, (st - 2) & 1, ab)) {
           ok = false;
           break;
         }
         tc_fence_after();
         const int n = min(kStepPages, n_cols - st * kStepPages);
         const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t k_addr = smem_u32(sKV + 2 * s * C::kTile);
+        const uint32_t k_addr = smem_u32(sK + ks * C::kTile);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
@@ -167,6 +172,7 @@ __global__ void __launch_bounds__(256, 1)
                   kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[b]);
+        umma_commit(&k_empty[ks]);
         if (st >= 1 && !issue_pv(st - 1)) ok = false;
       }
       if (ok && n_steps > 0) issue_pv(n_steps - 1);
@@ -182,12 +188,11 @@ __global__ void __launch_bounds__(256, 1)
     const int seg = code < 4 ? static_cast<int>(code) : -1;
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
+    uint32_t mw[4];
+    if (n_steps > 0) step_masks<kStepPages>(col_masks, wk.e0, min(kStepPages, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
-      const int n = min(kStepPages, n_cols - st * kStepPages);
-      const int N = 16 * n;
-      uint32_t mw[4];
-      step_masks(col_masks, wk.e0 + st * kStepPages, n, seg, mw);
+      const int N = 16 * min(kStepPages, n_cols - st * kStepPages);
       ok = mbar_wait(&s_full[b], (st >> 1) & 1, ab);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -196,26 +201,41 @@ __global__ void __launch_bounds__(256, 1)
 #pragma unroll
       for (int pc = 0; pc < 4; ++pc)
         if (pc * 32 < N) tmem_ld32(tmem + 128 * b + lane_off + pc * 32, sr[pc]);
+      // masks of the next step load while this one computes
+      uint32_t mw_next[4] = {0u, 0u, 0u, 0u};
+      if (st + 1 < n_steps)
+        step_masks<kStepPages>(col_masks, wk.e0 + (st + 1) * kStepPages,
+                               min(kStepPages, n_cols - (st + 1) * kStepPages), seg, mw_next);
       tmem_wait_ld();
       float mx = -INFINITY;
 #pragma unroll
       for (int pc = 0; pc < 4; ++pc) {
+        if (pc * 32 < N) {
+          if (mw[pc] == 0xFFFFFFFFu) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const bool on = (pc * 32 < N) && ((mw[pc] >> i) & 1u);
-          const float x = on ? __uint_as_float(sr[pc][i]) * sl2 : -INFINITY;
-          sr[pc][i] = __float_as_uint(x);
-          mx = fmaxf(mx, x);
+            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[pc][i]));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const float x = ((mw[pc] >> i) & 1u) ? __uint_as_float(sr[pc][i]) : -INFINITY;
+              sr[pc][i] = __float_as_uint(x);
+              mx = fmaxf(mx, x);
+            }
+          }
         }
       }
-      const bool resc = mx > m_used + kRescaleThreshold;
-      const float m_new = resc ? mx : m_used;
+      const float mx2 = mx * sl2;  // running max in log2 units (scale > 0)
+      const bool resc = mx2 > m_used + kRescaleThreshold;
+      const float m_new = resc ? mx2 : m_used;
       const float alpha = resc ? ex2(m_used - m_new) : 1.0f;
-      if (st > 0 && __any_sync(0xffffffffu, resc)) {
-        // O holds steps < st: wait for the last PV, then rescale this warp's rows
-        ok = mbar_wait(o_done, (st - 1) & 1, ab);
-        ok = __all_sync(0xffffffffu, ok);
+      if (st > 0) {
+        // Observe every PV completion in order (PV(st-1) here): a parity wait
+        // is only unambiguous while the barrier is at most one phase ahead.
+        ok = __all_sync(0xffffffffu, mbar_wait(o_done, (st - 1) & 1, ab));
         if (!ok) break;
+      }
+      if (st > 0 && __any_sync(0xffffffffu, resc)) {
+        // O holds steps < st: rescale this warp's rows
         tc_fence_after();
 #pragma unroll
         for (int pc = 0; pc < D / 32; ++pc) {
@@ -229,7 +249,7 @@ __global__ void __launch_bounds__(256, 1)
       }
       l *= alpha;
       m_used = m_new;
-      const float mu = (m_used == -INFINITY) ? 0.f : m_used;
+      const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
       float lsum = 0.f;
 #pragma unroll
       for (int pc = 0; pc < 4; ++pc) {
@@ -237,8 +257,8 @@ __global__ void __launch_bounds__(256, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(__uint_as_float(sr[pc][2 * i]) - mu);
-            const float p1 = ex2(__uint_as_float(sr[pc][2 * i + 1]) - mu);
+            const float p0 = ex2(fmaf(__uint_as_float(sr[pc][2 * i]), sl2, neg_mu));
+            const float p1 = ex2(fmaf(__uint_as_float(sr[pc][2 * i + 1]), sl2, neg_mu));
             lsum += p0 + p1;
             pk[i] = pack_bf16(p0, p1);
           }
@@ -249,6 +269,8 @@ __global__ void __launch_bounds__(256, 1)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) mw[i] = mw_next[i];
     }
     if (ok && n_steps > 0) {
       ok = mbar_wait(o_done, (n_steps - 1) & 1, ab);

@@ -306,6 +306,12 @@ void free_plan_device(spattn_plan_s* P) {
   cudaFree(P->d_k_invalid);
   cudaFree(P->d_err);
   cudaFree(P->d_delta);
+  for (auto& e : P->events) {
+    cudaEventDestroy(e.start);
+    cudaEventDestroy(e.stop);
+  }
+  P->events.clear();
+  P->n_events = 0;
 }
 
 int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) {
@@ -316,7 +322,7 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if (L->head_dim != 64 && L->head_dim != 128) return SPATTN_ERR_UNSUPPORTED;
   if (L->q_slots >= (int64_t(1) << 31) - 64 || L->kv_slots >= (int64_t(1) << 31) - 64) return SPATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(L->batch) * L->heads >= (int64_t(1) << 31)) return SPATTN_ERR_UNSUPPORTED;
-  if (!std::isfinite(L->scale)) return SPATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(L->scale) || L->scale < 0.f) return SPATTN_ERR_INVALID_ARG;
   if (G->row_ptr[static_cast<int64_t>(L->heads) * L->n_q_groups] > 0 && !G->kv_groups) return SPATTN_ERR_INVALID_ARG;
 
   P->batch = L->batch;

@@ -6,7 +6,9 @@
 #include <string>
 #include <vector>
 
-#include "../../include/spattn.h"
+#include <cuda_runtime.h>
+
+#include "spattn.h"
 
 namespace spattn {
 
@@ -75,4 +77,12 @@ struct spattn_plan_s {
   int64_t device_bytes = 0;
   double plan_ms = 0.0;
   std::vector<int32_t> scratch;  // buffer behind spattn_plan_pages / spattn_plan_qblocks
+  // per-kernel event record (spattn_profile)
+  bool profiling = false;
+  struct EventRec {
+    int kernel;
+    cudaEvent_t start, stop;
+  };
+  std::vector<EventRec> events;   // pool; the first n_events are in use
+  size_t n_events = 0;
 };

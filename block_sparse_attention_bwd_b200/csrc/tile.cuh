@@ -37,19 +37,32 @@ __device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {
   return x;
 }
 
-// Row mask of one step: bit c of word c/32 <=> column c of the step may be
-// attended by this row.  `seg` < 0 gives an all-zero mask.
+// Row mask of one step of NP pages: bit c of word c/32 <=> column c of the
+// step may be attended by this row.  `seg` < 0 gives an all-zero mask.
+template <int NP>
 __device__ __forceinline__ void step_masks(const uint64_t* __restrict__ masks, int first, int n, int seg,
-                                           uint32_t (&mw)[4]) {
+                                           uint32_t (&mw)[NP / 2]) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) mw[i] = 0u;
+  for (int i = 0; i < NP / 2; ++i) mw[i] = 0u;
   if (seg < 0) return;
 #pragma unroll
-  for (int j = 0; j < kStepPages; ++j) {
+  for (int j = 0; j < NP; ++j) {
     if (j < n) {
       const uint32_t bits = static_cast<uint32_t>(__ldg(masks + first + j) >> (16 * seg)) & 0xFFFFu;
       mw[j >> 1] |= bits << (16 * (j & 1));
     }
+  }
+}
+
+// TMA-load n 16-row pages (all 64-column chunks) into a stage whose chunks
+// are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every chunk.
+template <int NCH>
+__device__ __forceinline__ void load_pages(uint8_t* dst, int chunk_bytes, const CUtensorMap* map,
+                                           const int32_t* __restrict__ pages, int n, int bh, uint64_t* bar) {
+  for (int j = 0; j < n; ++j) {
+    const int row = __ldg(pages + j) * 16;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) tma_load_3d(dst + c * chunk_bytes + j * 2048, map, c * 64, row, bh, bar);
   }
 }
 

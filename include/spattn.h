@@ -69,7 +69,7 @@ typedef struct {
   const int32_t* q_group;         /* host [q_slots], -1 = padded */
   const int32_t* kv_group;        /* host [kv_slots], -1 = padded */
   int32_t n_q_groups, n_kv_groups;
-  float scale;                    /* softmax scale; 0 selects 1/sqrt(head_dim) */
+  float scale;                    /* softmax scale > 0; 0 selects 1/sqrt(head_dim) */
 } spattn_layout;
 
 typedef struct {
@@ -88,8 +88,24 @@ typedef struct {
   int64_t n_entries_fwd;         /* (work item, K page) entries of one batch */
   int64_t n_entries_dkdv;        /* (work item, Q page) entries of one batch */
   int64_t device_bytes;          /* device memory held by the plan */
+  int64_t launches_fwd;          /* kernels one spattn_fwd call launches */
+  int64_t launches_bwd;          /* kernels one spattn_bwd call launches */
   double plan_ms;                /* host time spent in spattn_plan */
 } spattn_stats;
+
+/* Kernel ids of spattn_kernel_times. */
+enum spattn_kernel {
+  SPATTN_K_FWD = 0,   /* forward attention (O, LSE) */
+  SPATTN_K_FILL = 1,  /* zero fill of pages without a valid slot */
+  SPATTN_K_DELTA = 2, /* rowsum(dO * O) */
+  SPATTN_K_DKDV = 3,  /* key-owned dK, dV */
+  SPATTN_K_DQ = 4     /* query-owned dQ */
+};
+
+typedef struct {
+  double ms[5];        /* device time per kernel id, summed over recorded launches */
+  int64_t launches[5]; /* recorded launches per kernel id */
+} spattn_kernel_times;
 
 /* Build a plan: validate layout and graph, find valid 16-row pages, pack
  * owned tiles, and build the per-tile page lists and masks for the forward /
@@ -115,6 +131,14 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
 int spattn_check(spattn_plan_t plan, void* stream);
 
 int spattn_plan_stats(spattn_plan_t plan, spattn_stats* stats);
+
+/* Per-kernel device timing.  While enabled, spattn_fwd / spattn_bwd record a
+ * CUDA event pair around every kernel they launch, on the launch stream.
+ * spattn_profile(plan, 1) starts recording, (plan, 0) stops; both discard
+ * what was recorded.  spattn_profile_read waits for the recorded events,
+ * returns their summed durations and clears the record. */
+int spattn_profile(spattn_plan_t plan, int enable);
+int spattn_profile_read(spattn_plan_t plan, spattn_kernel_times* out);
 
 /* Canonical page list of (head, Q block): ascending pages holding at least
  * one key that some query of the block may attend.  *pages points into a

@@ -13,6 +13,7 @@ from .configs import (  # noqa: F401
     Problem,
     make_problem,
     make_tensors,
+    with_heads,
     sta_layout,
     sta_graph,
     vsa_graph,

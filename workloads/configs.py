@@ -246,6 +246,15 @@ def make_problem(name: str) -> Problem:
     raise KeyError(name)
 
 
+def with_heads(problem: Problem, heads: int) -> Problem:
+    """The same layout with the graph of the first ``heads`` heads only."""
+    if not 1 <= heads <= problem.heads:
+        raise ValueError(f"heads must be in [1, {problem.heads}]")
+    end = problem.row_ptr[heads * problem.n_q_groups]
+    return dataclasses.replace(problem, heads=heads, row_ptr=problem.row_ptr[:heads * problem.n_q_groups + 1].copy(),
+                               kv_groups=problem.kv_groups[:end].copy())
+
+
 def make_tensors(problem: Problem, names: Sequence[str] = ("q", "k", "v", "do"),
                  batch: Optional[int] = None) -> Dict[str, "torch.Tensor"]:
     """Seeded bf16 tensors [B, H, S, D] on the CPU; padded slots hold the sentinel."""
