@@ -34,7 +34,7 @@ STATUS_NAMES = {
 }
 
 ENTRY_POINTS = (
-    "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_check", "spattn_plan_stats", "spattn_profile",
+    "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_bwd_noalloc", "spattn_check", "spattn_plan_stats", "spattn_profile",
     "spattn_profile_read", "spattn_plan_pages", "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy",
     "spattn_status_string",
 )
@@ -87,6 +87,7 @@ def _lib():
         lib.spattn_plan.argtypes = [ctypes.POINTER(_Layout), ctypes.POINTER(_Graph), ctypes.POINTER(P)]
         lib.spattn_fwd.argtypes = [P, P, P, P, P, P, P]
         lib.spattn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
+        lib.spattn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
         lib.spattn_check.argtypes = [P, P]
         lib.spattn_plan_stats.argtypes = [P, ctypes.POINTER(_Stats)]
         lib.spattn_plan_pages.argtypes = [P, I32, I64, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64)]

@@ -91,6 +91,15 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
 }
 
 }  // namespace
+
+// Entry points for other translation units of the library.
+bool make_tensor_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  return make_map(m, ptr, head_dim, rows, bh);
+}
+TileArgs make_tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots) {
+  return tile_args(P, w, own_slots, col_slots);
+}
+
 }  // namespace spattn
 
 using namespace spattn;

@@ -126,6 +126,21 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
 int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* d_o,
                spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream);
 
+/* Backward pass that allocates nothing, for callers that cannot allocate
+ * device memory when they run it (for example when another allocator has
+ * reserved the GPU, or under a fixed device-memory budget).  The paper has
+ * no counterpart; it is a deployment variant of spattn_bwd with the same
+ * arguments and results.  Its fp32 scratch (one value per query row) is a
+ * fixed static device array of 4,194,304 floats (16 MiB) that every GPU
+ * loading the library holds until exit, so batch * heads * q_slots must not
+ * exceed 4,194,304 (else SPATTN_ERR_UNSUPPORTED, nothing launched).  The
+ * first call on each device performs a one-time set-up (it looks up the
+ * array's device address) and should come before any stream capture.  All
+ * calls share the array and every call rewrites what it reads, so calls that
+ * overlap on the GPU (on different streams) race with each other. */
+int spattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                       const void* d_o, spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream);
+
 /* Synchronise `stream` and report (then clear) any device-side error the
  * plan's kernels recorded: SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_DEVICE. */
 int spattn_check(spattn_plan_t plan, void* stream);
