@@ -80,8 +80,14 @@ struct DkvCfg {
   static constexpr int kSmem = 2 * kTile + kQStages * kStageTile + kDStages * (kStageTile + kLdBytes) + 1024 + 512;
 };
 
+// 10 warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2..9 = two
+// groups of row threads; group g (warps 2+4g .. 5+4g) handles columns
+// 32g .. 32g+31 of every 64-column step (warp w reaches TMEM lanes of
+// quarter w%4).
+constexpr int kBwdThreads = 320;
+
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                 const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                 const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
@@ -134,7 +140,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&st_full[b], 1);
-      mbar_init(&pt_full[b], 128);
+      mbar_init(&pt_full[b], 256);
     }
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
@@ -148,52 +154,60 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tDV = tmem + 256, tDK = tmem + 256 + D;
 
   if (warp == 0) {
-    // ---------------- producer (lane 0: TMA; all lanes: LSE2 / Delta) ----------------
+    // ---------------- producer (whole warp) ----------------
+    // Lane j < n owns page j of a step: it holds the page id (fetched one step
+    // ahead) and issues that page's TMA boxes; every lane then fetches LSE2 and
+    // Delta for two of the step's 64 query columns.
     if (lane == 0) {
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
-      for (int p = 0; p < wk.n_own; ++p)
-        for (int c = 0; c < C::kNch; ++c) {
-          tma_load_3d(sK + c * kChunkBytes + p * 2048, &tm_k, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
-          tma_load_3d(sV + c * kChunkBytes + p * 2048, &tm_v, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
-        }
     }
+    __syncwarp();
+    if (lane < wk.n_own)
+#pragma unroll
+      for (int c = 0; c < C::kNch; ++c) {
+        tma_load_3d(sK + c * kChunkBytes + lane * 2048, &tm_k, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
+        tma_load_3d(sV + c * kChunkBytes + lane * 2048, &tm_v, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
+      }
+    int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int q_issued = 0, d_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
       const int qs = st % QS, ds = st % DS;
       const int n = min(NP, n_cols - st * NP);
-      const int32_t* pg = col_pages + wk.e0 + st * NP;
-      if (st >= QS) {
-        const bool ok = mbar_wait(&q_empty[qs], ((st / QS) - 1) & 1, ab);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&q_full[qs], n * C::kNch * 2048);
-        load_pages<C::kNch>(sQ + qs * C::kStageTile, kStageChunk, &tm_q, pg, n, wk.bh, &q_full[qs]);
-      }
+      const int pid = pid_next;
+      if (st + 1 < n_steps)
+        pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
+      if (st >= QS && !__all_sync(0xffffffffu, mbar_wait(&q_empty[qs], ((st / QS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&q_full[qs], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sQ + qs * C::kStageTile + c * kStageChunk + lane * 2048, &tm_q, c * 64, pid * 16, wk.bh, &q_full[qs]);
       q_issued = st + 1;
-      if (st >= DS) {
-        const bool ok = mbar_wait(&do_empty[ds], ((st / DS) - 1) & 1, ab);
-        if (!__all_sync(0xffffffffu, ok)) break;
-      }
-      if (lane == 0) {
-        mbar_arrive_expect_tx(&do_full[ds], n * C::kNch * 2048);
-        load_pages<C::kNch>(sDO + ds * C::kStageTile, kStageChunk, &tm_do, pg, n, wk.bh, &do_full[ds]);
-      }
+      if (st >= DS && !__all_sync(0xffffffffu, mbar_wait(&do_empty[ds], ((st / DS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&do_full[ds], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sDO + ds * C::kStageTile + c * kStageChunk + lane * 2048, &tm_do, c * 64, pid * 16, wk.bh,
+                      &do_full[ds]);
       d_issued = st + 1;
       float* sl = sLD + ds * 128;
-      for (int idx = lane; idx < 16 * NP; idx += 32) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int idx = lane + 32 * h;                     // column of the step
+        const int pg = __shfl_sync(0xffffffffu, pid, idx >> 4);
+        const int64_t slot = static_cast<int64_t>(pg) * 16 + (idx & 15);
         float l2 = 0.f, dl = 0.f;
-        if (idx < 16 * n) {
-          const int64_t slot = static_cast<int64_t>(__ldg(pg + (idx >> 4))) * 16 + (idx & 15);
-          if (slot < q_slots) {
-            const int64_t off = static_cast<int64_t>(wk.bh) * q_slots + slot;
-            l2 = __ldg(lse + off) * kLog2e;
-            dl = __ldg(delta + off);
-          }
+        if ((idx >> 4) < n && slot < q_slots) {
+          const int64_t off = static_cast<int64_t>(wk.bh) * q_slots + slot;
+          l2 = __ldg(lse + off) * kLog2e;
+          dl = __ldg(delta + off);
         }
         sl[idx] = l2;
         sl[64 + idx] = dl;
@@ -206,114 +220,123 @@ __global__ void __launch_bounds__(256, 1)
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t k_addr = smem_u32(sK), v_addr = smem_u32(sV);
-      const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
-      bool ok = mbar_wait(own_full, 0, ab);
+    // ---------------- MMA issuer (warp-wide; one elected lane issues) ----------------
+    const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
+    const uint64_t dqk = sdesc_sw128(smem_u32(sQ), 16, 1024);             // Q stages, K-major
+    const uint64_t ddk = sdesc_sw128(smem_u32(sDO), 16, 1024);            // dO stages, K-major
+    const uint64_t dqm = sdesc_sw128(smem_u32(sQ), kStageChunk, 1024);    // Q stages, MN-major
+    const uint64_t ddm = sdesc_sw128(smem_u32(sDO), kStageChunk, 1024);   // dO stages, MN-major
+    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
+    tc_fence_after();
+    auto issue_acc = [&](int st) -> bool {
+      const int b = st & 1, qs = st % QS, ds = st % DS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (st >> 1) & 1, ab))) return false;
       tc_fence_after();
-      auto issue_acc = [&](int st) -> bool {
-        const int b = st & 1, qs = st % QS, ds = st % DS;
-        if (!mbar_wait(&pt_full[b], (st >> 1) & 1, ab)) return false;
-        tc_fence_after();
-        const int n = min(NP, n_cols - st * NP);
-        const uint32_t q_addr = smem_u32(sQ + qs * C::kStageTile), do_addr = smem_u32(sDO + ds * C::kStageTile);
-        for (int j = 0; j < n; ++j)
-          umma_ts(tDV, tmem + 64 * b + 8 * j, sdesc_sw128(do_addr + j * 2048, kStageChunk, 1024), idesc_acc,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&do_empty[ds]);
-        for (int j = 0; j < n; ++j)
-          umma_ts(tDK, tmem + 128 + 64 * b + 8 * j, sdesc_sw128(q_addr + j * 2048, kStageChunk, 1024), idesc_acc,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&q_empty[qs]);
-        umma_commit(acc_step);
-        return true;
-      };
-      for (int st = 0; ok && st < n_steps; ++st) {
-        const int b = st & 1, qs = st % QS, ds = st % DS;
-        const int n = min(NP, n_cols - st * NP);
-        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t q_addr = smem_u32(sQ + qs * C::kStageTile), do_addr = smem_u32(sDO + ds * C::kStageTile);
-        // buffers b still feed dV(st-2) / dK(st-2) as TMEM A operands
-        if (st >= 2 && !mbar_wait(acc_step, (st - 2) & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(&q_full[qs], (st / QS) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
+      const int n = min(NP, n_cols - st * NP);
+      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile), bd = sdesc_add(ddm, ds * C::kStageTile);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + 64 * b, sdesc_sw128(k_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(q_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
-        }
-        if (!mbar_wait(&do_full[ds], (st / DS) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
+      for (int j = 0; j < NP; ++j)
+        if (j < n) umma_ts_w(tDV, tmem + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&do_empty[ds]);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          umma_ss(tmem + 128 + 64 * b, sdesc_sw128(v_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(do_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
-        }
-        umma_commit(&st_full[b]);
-        if (st >= 1 && !issue_acc(st - 1)) ok = false;
-      }
-      if (ok && n_steps > 0 && issue_acc(n_steps - 1)) umma_commit(acc_done);
-      umma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      for (int j = 0; j < NP; ++j)
+        if (j < n)
+          umma_ts_w(tDK, tmem + 128 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&q_empty[qs]);
+      umma_commit_w(acc_step);
+      return true;
+    };
+    for (int st = 0; ok && st < n_steps; ++st) {
+      const int b = st & 1, qs = st % QS, ds = st % DS;
+      const int n = min(NP, n_cols - st * NP);
+      const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+      // buffers b still feed dV(st-2) / dK(st-2) as TMEM A operands
+      bool w = (st < 2 || mbar_wait(acc_step, (st - 2) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile), bd = sdesc_add(ddk, ds * C::kStageTile);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_ss_w(tmem + 64 * b, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                  sdesc_add(bq, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (st / DS) & 1, ab))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_ss_w(tmem + 128 + 64 * b, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                  sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      umma_commit_w(&st_full[b]);
+      if (st >= 1 && !issue_acc(st - 1)) ok = false;
     }
-  } else if (warp >= 4) {
+    if (ok && n_steps > 0 && issue_acc(n_steps - 1)) umma_commit_w(acc_done);
+    umma_commit_w(drain);
+    mbar_wait_drain(drain, 0);
+  } else {
     // ---------------- P^T, dS^T (one key row per thread) + epilogue ----------------
-    const int q4 = warp - 4;
+    const int grp = (warp - 2) >> 2;  // column half of each step
+    const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
     const int seg = code < 4 ? static_cast<int>(code) : -1;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
     uint32_t mw[2];
     if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1, ds = st % DS;
       const int N = 16 * min(NP, n_cols - st * NP);
+      const bool active = grp * 32 < N;
       ok = mbar_wait(&st_full[b], (st >> 1) & 1, ab) && mbar_wait(&ld_full[ds], (st / DS) & 1, ab);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      uint32_t a[2][32], d[2][32];
-#pragma unroll
-      for (int pc = 0; pc < 2; ++pc)
-        if (pc * 32 < N) {
-          tmem_ld32(tmem + 64 * b + lane_off + pc * 32, a[pc]);
-          tmem_ld32(tmem + 128 + 64 * b + lane_off + pc * 32, d[pc]);
-        }
+      uint32_t a[32], d[32];
+      if (active) {
+        tmem_ld32(tmem + 64 * b + lane_off + grp * 32, a);
+        tmem_ld32(tmem + 128 + 64 * b + lane_off + grp * 32, d);
+      }
       uint32_t mw_next[2] = {0u, 0u};
       if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
-      tmem_wait_ld();
-      const float4* sl4 = reinterpret_cast<const float4*>(sLD + ds * 128);
+      if (active) {
+        tmem_wait_ld();
+        const uint32_t m = grp ? mw[1] : mw[0];
+        const float4* sl4 = reinterpret_cast<const float4*>(sLD + ds * 128 + grp * 32);
+        const float4* sd4 = reinterpret_cast<const float4*>(sLD + ds * 128 + 64 + grp * 32);
+        uint32_t pp[16], pd[16];
 #pragma unroll
-      for (int pc = 0; pc < 2; ++pc) {
-        if (pc * 32 < N) {
-          uint32_t pp[16], pd[16];
+        for (int i4 = 0; i4 < 8; ++i4) {
+          const float4 L = sl4[i4];
+          const float4 Dl = sd4[i4];
+          float x0, x1, x2, x3;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
+                           f2_pack(-L.x, -L.y)), x0, x1);
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
+                           f2_pack(-L.z, -L.w)), x2, x3);
+          float p[4] = {ex2(x0), ex2(x1), ex2(x2), ex2(x3)};
 #pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 L = sl4[pc * 8 + i4];
-            const float4 Dl = sl4[16 + pc * 8 + i4];
-            const float lv[4] = {L.x, L.y, L.z, L.w};
-            const float dv[4] = {Dl.x, Dl.y, Dl.z, Dl.w};
-            float pv[4], sv[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int i = 4 * i4 + h;
-              const bool on = (mw[pc] >> i) & 1u;
-              const float p = on ? ex2(fmaf(__uint_as_float(a[pc][i]), sl2, -lv[h])) : 0.f;
-              pv[h] = p;
-              sv[h] = on ? p * (__uint_as_float(d[pc][i]) - dv[h]) : 0.f;
-            }
-            pp[2 * i4] = pack_bf16(pv[0], pv[1]);
-            pp[2 * i4 + 1] = pack_bf16(pv[2], pv[3]);
-            pd[2 * i4] = pack_bf16(sv[0], sv[1]);
-            pd[2 * i4 + 1] = pack_bf16(sv[2], sv[3]);
-          }
-          tmem_st16(tmem + 64 * b + lane_off + pc * 16, pp);
-          tmem_st16(tmem + 128 + 64 * b + lane_off + pc * 16, pd);
+          for (int h = 0; h < 4; ++h)
+            if (!((m >> (4 * i4 + h)) & 1u)) p[h] = 0.f;
+          float g0, g1, g2, g3;
+          f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])), f2_pack(-Dl.x, -Dl.y)),
+                    g0, g1);
+          f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
+                           f2_pack(-Dl.z, -Dl.w)), g2, g3);
+          float s0, s1, s2, s3;
+          f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_pack(g0, g1)), s0, s1);
+          f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_pack(g2, g3)), s2, s3);
+          pp[2 * i4] = pack_bf16(p[0], p[1]);
+          pp[2 * i4 + 1] = pack_bf16(p[2], p[3]);
+          // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
+          pd[2 * i4] = pack_bf16(p[0] != 0.f ? s0 : 0.f, p[1] != 0.f ? s1 : 0.f);
+          pd[2 * i4 + 1] = pack_bf16(p[2] != 0.f ? s2 : 0.f, p[3] != 0.f ? s3 : 0.f);
         }
+        tmem_st16(tmem + 64 * b + lane_off + grp * 16, pp);
+        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 16, pd);
+        tmem_wait_st();
       }
-      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&pt_full[b]);
       mw[0] = mw_next[0];
@@ -324,27 +347,22 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
     }
     if (ok) {
+      // group 0 writes dV, group 1 writes scale * dK
       const bool owned = code != 15u && row < 16 * wk.n_own;
       const int64_t slot = owned ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
       const bool write = owned && slot < kv_slots;
       const int64_t base = (static_cast<int64_t>(wk.bh) * kv_slots + slot) * D;
+      const uint32_t tacc = grp == 0 ? tDV : tDK;
+      __nv_bfloat16* out = grp == 0 ? out_dv : out_dk;
+      const float mul = grp == 0 ? 1.0f : scale;
 #pragma unroll
       for (int pc = 0; pc < D / 32; ++pc) {
         uint32_t r[32] = {};
         if (n_steps > 0) {
-          tmem_ld32(tDV + lane_off + pc * 32, r);
+          tmem_ld32(tacc + lane_off + pc * 32, r);
           tmem_wait_ld();
         }
-        if (write) store_row32(out_dv + base + pc * 32, r, 1.0f, n_steps == 0);
-      }
-#pragma unroll
-      for (int pc = 0; pc < D / 32; ++pc) {
-        uint32_t r[32] = {};
-        if (n_steps > 0) {
-          tmem_ld32(tDK + lane_off + pc * 32, r);
-          tmem_wait_ld();
-        }
-        if (write) store_row32(out_dk + base + pc * 32, r, scale, n_steps == 0);
+        if (write) store_row32(out + base + pc * 32, r, mul, n_steps == 0);
       }
     }
   }
@@ -373,7 +391,7 @@ struct DqCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
               const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
               const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
@@ -420,7 +438,7 @@ __global__ void __launch_bounds__(256, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sd_full[b], 1);
-      mbar_init(&ds_full[b], 128);
+      mbar_init(&ds_full[b], 256);
     }
     mbar_init(acc_done, 1);
     mbar_init(dq_step, 1);
@@ -435,83 +453,103 @@ __global__ void __launch_bounds__(256, 1)
   const uint32_t tDQ = tmem + 256;
 
   if (warp == 0) {
+    // ---------------- producer (whole warp; lane j owns page j of a step) ----------------
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
-      for (int p = 0; p < wk.n_own; ++p)
-        for (int c = 0; c < C::kNch; ++c) {
-          tma_load_3d(sQ + c * kChunkBytes + p * 2048, &tm_q, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
-          tma_load_3d(sDO + c * kChunkBytes + p * 2048, &tm_do, c * 64, wk.own_page(p) * 16, wk.bh, own_full);
-        }
-      int k_issued = 0, v_issued = 0;
-      for (int st = 0; st < n_steps; ++st) {
-        const int ks = st % KS, vs = st % VS;
-        const int n = min(NP, n_cols - st * NP);
-        const int32_t* pg = col_pages + wk.e0 + st * NP;
-        if (st >= KS && !mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
-        load_pages<C::kNch>(sK + ks * C::kStageTile, kStageChunk, &tm_k, pg, n, wk.bh, &k_full[ks]);
-        k_issued = st + 1;
-        if (st >= VS && !mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
-        load_pages<C::kNch>(sV + vs * C::kStageTile, kStageChunk, &tm_v, pg, n, wk.bh, &v_full[vs]);
-        v_issued = st + 1;
+    }
+    __syncwarp();
+    if (lane < wk.n_own)
+#pragma unroll
+      for (int c = 0; c < C::kNch; ++c) {
+        tma_load_3d(sQ + c * kChunkBytes + lane * 2048, &tm_q, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
+        tma_load_3d(sDO + c * kChunkBytes + lane * 2048, &tm_do, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
       }
+    int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
+    int k_issued = 0, v_issued = 0;
+    for (int st = 0; st < n_steps; ++st) {
+      const int ks = st % KS, vs = st % VS;
+      const int n = min(NP, n_cols - st * NP);
+      const int pid = pid_next;
+      if (st + 1 < n_steps)
+        pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
+      if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sK + ks * C::kStageTile + c * kStageChunk + lane * 2048, &tm_k, c * 64, pid * 16, wk.bh, &k_full[ks]);
+      k_issued = st + 1;
+      if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sV + vs * C::kStageTile + c * kStageChunk + lane * 2048, &tm_v, c * 64, pid * 16, wk.bh, &v_full[vs]);
+      v_issued = st + 1;
+    }
+    if (lane == 0) {
       for (int st = max(0, k_issued - KS); st < k_issued; ++st) mbar_wait_drain(&k_full[st % KS], (st / KS) & 1);
       for (int st = max(0, v_issued - VS); st < v_issued; ++st) mbar_wait_drain(&v_full[st % VS], (st / VS) & 1);
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t q_addr = smem_u32(sQ), do_addr = smem_u32(sDO);
-      const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
-      bool ok = mbar_wait(own_full, 0, ab);
+    // ---------------- MMA issuer (warp-wide; one elected lane issues) ----------------
+    const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t ddo0 = sdesc_sw128(smem_u32(sDO), 16, 1024);
+    const uint64_t dkk = sdesc_sw128(smem_u32(sK), 16, 1024);            // K stages, K-major
+    const uint64_t dkm = sdesc_sw128(smem_u32(sK), kStageChunk, 1024);   // K stages, MN-major
+    const uint64_t dvk = sdesc_sw128(smem_u32(sV), 16, 1024);            // V stages, K-major
+    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
+    tc_fence_after();
+    auto issue_dq = [&](int st) -> bool {
+      const int b = st & 1, ks = st % KS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[b], (st >> 1) & 1, ab))) return false;
       tc_fence_after();
-      auto issue_dq = [&](int st) -> bool {
-        const int b = st & 1, ks = st % KS;
-        if (!mbar_wait(&ds_full[b], (st >> 1) & 1, ab)) return false;
-        tc_fence_after();
-        const int n = min(NP, n_cols - st * NP);
-        const uint32_t k_addr = smem_u32(sK + ks * C::kStageTile);
-        for (int j = 0; j < n; ++j)
-          umma_ts(tDQ, tmem + 64 * b + 8 * j, sdesc_sw128(k_addr + j * 2048, kStageChunk, 1024), idesc_acc,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&k_empty[ks]);
-        umma_commit(dq_step);
-        return true;
-      };
-      for (int st = 0; ok && st < n_steps; ++st) {
-        const int b = st & 1, ks = st % KS, vs = st % VS;
-        const int n = min(NP, n_cols - st * NP);
-        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t k_addr = smem_u32(sK + ks * C::kStageTile), v_addr = smem_u32(sV + vs * C::kStageTile);
-        // buffer b still feeds dQ(st-2) as its TMEM A operand
-        if (st >= 2 && !mbar_wait(dq_step, (st - 2) & 1, ab)) { ok = false; break; }
-        if (!mbar_wait(&k_full[ks], (st / KS) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
+      const int n = min(NP, n_cols - st * NP);
+      const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + 64 * b, sdesc_sw128(q_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(k_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
-        if (!mbar_wait(&v_full[vs], (st / VS) & 1, ab)) { ok = false; break; }
-        tc_fence_after();
+      for (int j = 0; j < NP; ++j)
+        if (j < n) umma_ts_w(tDQ, tmem + 64 * b + 8 * j, sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&k_empty[ks]);
+      umma_commit_w(dq_step);
+      return true;
+    };
+    for (int st = 0; ok && st < n_steps; ++st) {
+      const int b = st & 1, ks = st % KS, vs = st % VS;
+      const int n = min(NP, n_cols - st * NP);
+      const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+      // buffer b still feeds dQ(st-2) as its TMEM A operand
+      bool w = (st < 2 || mbar_wait(dq_step, (st - 2) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+      tc_fence_after();
+      const uint64_t bk = sdesc_add(dkk, ks * C::kStageTile), bv = sdesc_add(dvk, vs * C::kStageTile);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk)
-          umma_ss(tmem + 128 + 64 * b, sdesc_sw128(do_addr + (kk >> 2) * kChunkBytes + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(v_addr + (kk >> 2) * kStageChunk + (kk & 3) * 32, 16, 1024), idesc_s, kk > 0);
-        umma_commit(&v_empty[vs]);
-        umma_commit(&sd_full[b]);
-        if (st >= 1 && !issue_dq(st - 1)) ok = false;
-      }
-      if (ok && n_steps > 0 && issue_dq(n_steps - 1)) umma_commit(acc_done);
-      umma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_ss_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                  sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (st / VS) & 1, ab))) { ok = false; break; }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_ss_w(tmem + 128 + 64 * b, sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                  sdesc_add(bv, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      umma_commit_w(&v_empty[vs]);
+      umma_commit_w(&sd_full[b]);
+      if (st >= 1 && !issue_dq(st - 1)) ok = false;
     }
-  } else if (warp >= 4) {
-    const int q4 = warp - 4;
+    if (ok && n_steps > 0 && issue_dq(n_steps - 1)) umma_commit_w(acc_done);
+    umma_commit_w(drain);
+    mbar_wait_drain(drain, 0);
+  } else {
+    const int grp = (warp - 2) >> 2;  // column half of each step
+    const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
@@ -522,44 +560,45 @@ __global__ void __launch_bounds__(256, 1)
     const int64_t roff = static_cast<int64_t>(wk.bh) * q_slots + slot;
     const float lse2 = (valid_slot && seg >= 0) ? __ldg(lse + roff) * kLog2e : 0.f;
     const float dl = (valid_slot && seg >= 0) ? __ldg(delta + roff) : 0.f;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    const uint64_t nl2 = f2_pack(-lse2, -lse2);
+    const uint64_t ndl = f2_pack(-dl, -dl);
     bool ok = true;
     uint32_t mw[2];
     if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
+      const bool active = grp * 32 < N;
       ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
-      uint32_t a[2][32], d[2][32];
-#pragma unroll
-      for (int pc = 0; pc < 2; ++pc)
-        if (pc * 32 < N) {
-          tmem_ld32(tmem + 64 * b + lane_off + pc * 32, a[pc]);
-          tmem_ld32(tmem + 128 + 64 * b + lane_off + pc * 32, d[pc]);
-        }
+      uint32_t a[32], d[32];
+      if (active) {
+        tmem_ld32(tmem + 64 * b + lane_off + grp * 32, a);
+        tmem_ld32(tmem + 128 + 64 * b + lane_off + grp * 32, d);
+      }
       uint32_t mw_next[2] = {0u, 0u};
       if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
-      tmem_wait_ld();
+      if (active) {
+        tmem_wait_ld();
+        const uint32_t m = grp ? mw[1] : mw[0];
+        uint32_t pd[16];
 #pragma unroll
-      for (int pc = 0; pc < 2; ++pc) {
-        if (pc * 32 < N) {
-          uint32_t pd[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float sv[2];
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const bool on = (mw[pc] >> (2 * i + h)) & 1u;
-              const float p = on ? ex2(fmaf(__uint_as_float(a[pc][2 * i + h]), sl2, -lse2)) : 0.f;
-              sv[h] = on ? p * (__uint_as_float(d[pc][2 * i + h]) - dl) : 0.f;
-            }
-            pd[i] = pack_bf16(sv[0], sv[1]);
-          }
-          tmem_st16(tmem + 64 * b + lane_off + pc * 16, pd);
+        for (int i = 0; i < 16; ++i) {
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2, nl2), x0, x1);
+          float p0 = ex2(x0), p1 = ex2(x1);
+          if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
+          if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
+          float g0, g1;
+          f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), ndl)),
+                    g0, g1);
+          pd[i] = pack_bf16(p0 != 0.f ? g0 : 0.f, p1 != 0.f ? g1 : 0.f);
         }
+        tmem_st16(tmem + 64 * b + lane_off + grp * 16, pd);
+        tmem_wait_st();
       }
-      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&ds_full[b]);
       mw[0] = mw_next[0];
@@ -570,15 +609,17 @@ __global__ void __launch_bounds__(256, 1)
       tc_fence_after();
     }
     if (ok) {
+      // group g writes columns [g*D/2, (g+1)*D/2) of dQ
       __nv_bfloat16* dst = out_dq + roff * D;
 #pragma unroll
-      for (int pc = 0; pc < D / 32; ++pc) {
+      for (int pc = 0; pc < D / 64; ++pc) {
+        const int col = grp * (D / 2) + pc * 32;
         uint32_t r[32] = {};
         if (n_steps > 0) {
-          tmem_ld32(tDQ + lane_off + pc * 32, r);
+          tmem_ld32(tDQ + lane_off + col, r);
           tmem_wait_ld();
         }
-        if (valid_slot) store_row32(dst + pc * 32, r, scale, n_steps == 0);
+        if (valid_slot) store_row32(dst + col, r, scale, n_steps == 0);
       }
     }
   }
@@ -612,7 +653,7 @@ static cudaError_t launch_dkdv_t(const CUtensorMap& tk, const CUtensorMap& tv, c
   using C = DkvCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
-  dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), 256, C::kSmem, st>>>(
+  dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), kBwdThreads, C::kSmem, st>>>(
       tk, tv, tq, tdo, a.work, a.pages, a.masks, lse, delta, dk, dv, a.own_slots, a.col_slots, a.scale * kLog2e,
       a.scale, a.err);
   return cudaGetLastError();
@@ -625,7 +666,7 @@ static cudaError_t launch_dq_t(const CUtensorMap& tq, const CUtensorMap& tdo, co
   using C = DqCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
-  dq_kernel<D><<<static_cast<unsigned>(a.n_work), 256, C::kSmem, st>>>(
+  dq_kernel<D><<<static_cast<unsigned>(a.n_work), kBwdThreads, C::kSmem, st>>>(
       tq, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.err);
   return cudaGetLastError();
 }

@@ -26,34 +26,45 @@ namespace {
 
 using namespace dev;
 
+// 64 key columns (4 pages) per step; two CTAs share an SM (256 TMEM columns
+// and < 113 KB of shared memory each), so the row threads of one CTA compute
+// while the tensor core runs the other CTA's MMAs.
+constexpr int kFwdStepPages = 4;
+constexpr int kFwdStageChunk = 64 * 128;  // one 64-column chunk of a 64-row stage
+
 template <int D>
 struct FwdCfg {
-  static constexpr int kNch = D / 64;                  // 64-column chunks
-  static constexpr int kTile = kNch * kChunkBytes;     // one 128-row operand
-  static constexpr int kKStages = (D == 128) ? 3 : 6;  // K ring depth
-  static constexpr int kVStages = (D == 128) ? 3 : 6;  // V ring depth
-  static constexpr int kSmem = kTile * (1 + kKStages + kVStages) + 1024 + 512;
+  static constexpr int kNch = D / 64;                     // 64-column chunks
+  static constexpr int kTile = kNch * kChunkBytes;        // 128-row query tile
+  static constexpr int kStage = kNch * kFwdStageChunk;    // 64-row K or V stage
+  static constexpr int kKStages = (D == 128) ? 2 : 4;     // K ring depth
+  static constexpr int kVStages = (D == 128) ? 2 : 4;     // V ring depth
+  static constexpr int kSmem = kTile + (kKStages + kVStages) * kStage + 1024 + 512;
 };
 
 // Rescale O only when the running max grows by more than 2^8 (log2 units):
 // P stays below 256 and the final O / l is unchanged.
 constexpr float kRescaleThreshold = 8.0f;
 
+// 6 warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2..5 = row
+// threads (warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31).
+constexpr int kFwdThreads = 192;
+
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kFwdThreads, 2)
     fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ work,
                const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
                __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
                int* err) {
   using C = FwdCfg<D>;
-  constexpr int KS = C::kKStages, VS = C::kVStages;
+  constexpr int KS = C::kKStages, VS = C::kVStages, NP = kFwdStepPages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::kTile;          // K stage s at sK + s*kTile
-  uint8_t* sV = sK + KS * C::kTile;       // V stage s at sV + s*kTile
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kTile);
+  uint8_t* sK = smem + C::kTile;          // K stage s at sK + s*kStage
+  uint8_t* sV = sK + KS * C::kStage;      // V stage s at sV + s*kStage
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kStage);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
   uint64_t* k_empty = k_full + KS;
@@ -69,7 +80,7 @@ __global__ void __launch_bounds__(256, 1)
 
   const Work wk = load_work(work, blockIdx.x);
   const int n_cols = wk.e1 - wk.e0;
-  const int n_steps = (n_cols + kStepPages - 1) / kStepPages;
+  const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
@@ -91,186 +102,207 @@ __global__ void __launch_bounds__(256, 1)
     mbar_init(drain, 1);
     fence_barrier_init();
   }
-  if (warp == 1) tmem_alloc(tslot, 512);
+  if (warp == 1) tmem_alloc(tslot, 256);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tO = tmem + 256;  // S buffers at columns 0 and 128
+  const uint32_t tO = tmem + 128;  // S buffers at columns 0 and 64
 
   if (warp == 0) {
+    // ---------------- producer (whole warp): K runs ahead of V ----------------
+    // Lane j < n owns page j of a step: it holds the page id (fetched one step
+    // ahead) and issues that page's TMA boxes.
     if (lane == 0) {
-      // ---------------- producer: K runs ahead of V ----------------
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       mbar_arrive_expect_tx(q_full, wk.n_own * C::kNch * 2048);
-      for (int p = 0; p < wk.n_own; ++p)
+    }
+    __syncwarp();
+    if (lane < wk.n_own)
+#pragma unroll
+      for (int c = 0; c < C::kNch; ++c)
+        tma_load_3d(sQ + c * kChunkBytes + lane * 2048, &tm_q, c * 64, wk.own_page(lane) * 16, wk.bh, q_full);
+    int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
+    int k_issued = 0, v_issued = 0;
+    for (int st = 0; st < n_steps; ++st) {
+      const int n = min(NP, n_cols - st * NP);
+      const int pid = pid_next;
+      if (st + 1 < n_steps)
+        pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
+      const int ks = st % KS, vs = st % VS;
+      if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
         for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sQ + c * kChunkBytes + p * 2048, &tm_q, c * 64, wk.own_page(p) * 16, wk.bh, q_full);
-      int k_issued = 0, v_issued = 0;
-      for (int st = 0; st < n_steps; ++st) {
-        const int n = min(kStepPages, n_cols - st * kStepPages);
-        const int32_t* pg = col_pages + wk.e0 + st * kStepPages;
-        const int ks = st % KS, vs = st % VS;
-        if (st >= KS && !mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
-        load_pages<C::kNch>(sK + ks * C::kTile, kChunkBytes, &tm_k, pg, n, wk.bh, &k_full[ks]);
-        k_issued = st + 1;
-        if (st >= VS && !mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab)) break;
-        mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
-        load_pages<C::kNch>(sV + vs * C::kTile, kChunkBytes, &tm_v, pg, n, wk.bh, &v_full[vs]);
-        v_issued = st + 1;
-      }
-      // no copy may still be landing in shared memory when the CTA exits
+          tma_load_3d(sK + ks * C::kStage + c * kFwdStageChunk + lane * 2048, &tm_k, c * 64, pid * 16, wk.bh, &k_full[ks]);
+      k_issued = st + 1;
+      if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
+      __syncwarp();
+      if (lane < n)
+#pragma unroll
+        for (int c = 0; c < C::kNch; ++c)
+          tma_load_3d(sV + vs * C::kStage + c * kFwdStageChunk + lane * 2048, &tm_v, c * 64, pid * 16, wk.bh, &v_full[vs]);
+      v_issued = st + 1;
+    }
+    // no copy may still be landing in shared memory when the CTA exits
+    if (lane == 0) {
       for (int st = max(0, k_issued - KS); st < k_issued; ++st) mbar_wait_drain(&k_full[st % KS], (st / KS) & 1);
       for (int st = max(0, v_issued - VS); st < v_issued; ++st) mbar_wait_drain(&v_full[st % VS], (st / VS) & 1);
       mbar_wait_drain(q_full, 0);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t idesc_pv = idesc_bf16(128, D, false, true);
-      bool ok = mbar_wait(q_full, 0, ab);
+    // ---------------- MMA issuer (warp-wide; one elected lane issues) ----------------
+    const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
+    const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kFwdStageChunk, 1024);
+    const uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+    bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, ab));
+    tc_fence_after();
+    auto issue_pv = [&](int st) -> bool {
+      const int b = st & 1, vs = st % VS;
+      const bool w = mbar_wait(&p_full[b], (st >> 1) & 1, ab) && mbar_wait(&v_full[vs], (st / VS) & 1, ab);
+      if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
-      auto issue_pv = [&](int st) -> bool {
-        const int b = st & 1, vs = st % VS;
-        if (!mbar_wait(&p_full[b], (st >> 1) & 1, ab)) return false;
-        if (!mbar_wait(&v_full[vs], (st / VS) & 1, ab)) return false;
-        tc_fence_after();
-        const int n = min(kStepPages, n_cols - st * kStepPages);
-        const uint32_t v_addr = smem_u32(sV + vs * C::kTile);
-        for (int j = 0; j < n; ++j)
-          umma_ts(tO, tmem + 128 * b + 8 * j, sdesc_sw128(v_addr + j * 2048, kChunkBytes, 1024), idesc_pv,
-                  (st > 0 || j > 0) ? 1u : 0u);
-        umma_commit(&v_empty[vs]);
-        umma_commit(o_done);
-        return true;
-      };
-      for (int st = 0; ok && st < n_steps; ++st) {
-        const int ks = st % KS, b = st & 1;
-        if (!mbar_wait(&k_full[ks], (st / KS) & 1, ab)) {
-          ok = false;
-          break;
-        }
-        // buffer b still holds P(st-2), the TMEM A operand of PV(st-2); let
-        // that MMA finish before S(st) overwrites it (waited every step, in
-        // order, so the parity is unambiguous)
-        if (st >= 2 && !mbar_wait(o_done, (st - 2) & 1, ab)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const int n = min(kStepPages, n_cols - st * kStepPages);
-        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-        const uint32_t k_addr = smem_u32(sK + ks * C::kTile);
+      const int n = min(NP, n_cols - st * NP);
+      const uint64_t dv = sdesc_add(dv0, vs * C::kStage);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-          umma_ss(tmem + 128 * b, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s,
-                  kk > 0 ? 1u : 0u);
-        }
-        umma_commit(&s_full[b]);
-        umma_commit(&k_empty[ks]);
-        if (st >= 1 && !issue_pv(st - 1)) ok = false;
+      for (int j = 0; j < NP; ++j)
+        if (j < n)
+          umma_ts_w(tO, tmem + 64 * b + 8 * j, sdesc_add(dv, j * 2048), idesc_pv, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&v_empty[vs]);
+      umma_commit_w(o_done);
+      return true;
+    };
+    for (int st = 0; ok && st < n_steps; ++st) {
+      const int ks = st % KS, b = st & 1;
+      // buffer b still holds P(st-2), the TMEM A operand of PV(st-2); let
+      // that MMA finish before S(st) overwrites it (waited every step, in
+      // order, so the parity is unambiguous)
+      const bool w = mbar_wait(&k_full[ks], (st / KS) & 1, ab) && (st < 2 || mbar_wait(o_done, (st - 2) & 1, ab));
+      if (!__all_sync(0xffffffffu, w)) {
+        ok = false;
+        break;
       }
-      if (ok && n_steps > 0) issue_pv(n_steps - 1);
-      umma_commit(drain);
-      mbar_wait_drain(drain, 0);
+      tc_fence_after();
+      const int n = min(NP, n_cols - st * NP);
+      const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+      const uint64_t dk = sdesc_add(dk0, ks * C::kStage);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk)
+        umma_ss_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                  sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
+      umma_commit_w(&s_full[b]);
+      umma_commit_w(&k_empty[ks]);
+      if (st >= 1 && !issue_pv(st - 1)) ok = false;
     }
-  } else if (warp >= 4) {
+    if (ok && n_steps > 0) issue_pv(n_steps - 1);
+    umma_commit_w(drain);
+    mbar_wait_drain(drain, 0);
+  } else {
     // ---------------- softmax + epilogue (one row per thread) ----------------
-    const int q4 = warp - 4;
+    const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
     const int seg = code < 4 ? static_cast<int>(code) : -1;
+    const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t mw[4];
-    if (n_steps > 0) step_masks<kStepPages>(col_masks, wk.e0, min(kStepPages, n_cols), seg, mw);
+    uint32_t mw[2];
+    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
-      const int N = 16 * min(kStepPages, n_cols - st * kStepPages);
-      ok = mbar_wait(&s_full[b], (st >> 1) & 1, ab);
-      ok = __all_sync(0xffffffffu, ok);
+      const int N = 16 * min(NP, n_cols - st * NP);
+      ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[2][32];
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc)
-        if (pc * 32 < N) tmem_ld32(tmem + 128 * b + lane_off + pc * 32, sr[pc]);
+      for (int pc = 0; pc < 2; ++pc)
+        if (pc * 32 < N) tmem_ld32(tmem + 64 * b + lane_off + pc * 32, sr[pc]);
       // masks of the next step load while this one computes
-      uint32_t mw_next[4] = {0u, 0u, 0u, 0u};
-      if (st + 1 < n_steps)
-        step_masks<kStepPages>(col_masks, wk.e0 + (st + 1) * kStepPages,
-                               min(kStepPages, n_cols - (st + 1) * kStepPages), seg, mw_next);
+      uint32_t mw_next[2] = {0u, 0u};
+      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
       tmem_wait_ld();
-      float mx = -INFINITY;
+      // masked row max over four independent chains
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
+      for (int pc = 0; pc < 2; ++pc) {
         if (pc * 32 < N) {
-          if (mw[pc] == 0xFFFFFFFFu) {
+          if (mw[pc] != 0xFFFFFFFFu) {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) mx = fmaxf(mx, __uint_as_float(sr[pc][i]));
-          } else {
+            for (int i = 0; i < 32; ++i)
+              if (!((mw[pc] >> i) & 1u)) sr[pc][i] = 0xFF800000u;  // -inf
+          }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const float x = ((mw[pc] >> i) & 1u) ? __uint_as_float(sr[pc][i]) : -INFINITY;
-              sr[pc][i] = __float_as_uint(x);
-              mx = fmaxf(mx, x);
-            }
+          for (int i = 0; i < 32; i += 8) {
+            mx[0] = fmax3(mx[0], __uint_as_float(sr[pc][i]), __uint_as_float(sr[pc][i + 1]));
+            mx[1] = fmax3(mx[1], __uint_as_float(sr[pc][i + 2]), __uint_as_float(sr[pc][i + 3]));
+            mx[2] = fmax3(mx[2], __uint_as_float(sr[pc][i + 4]), __uint_as_float(sr[pc][i + 5]));
+            mx[3] = fmax3(mx[3], __uint_as_float(sr[pc][i + 6]), __uint_as_float(sr[pc][i + 7]));
           }
         }
       }
-      const float mx2 = mx * sl2;  // running max in log2 units (scale > 0)
+      const float mx2 = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3])) * sl2;  // log2 units (scale > 0)
       const bool resc = mx2 > m_used + kRescaleThreshold;
       const float m_new = resc ? mx2 : m_used;
       const float alpha = resc ? ex2(m_used - m_new) : 1.0f;
+      l *= alpha;
+      m_used = m_new;
+      const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
+      const uint64_t nmu2 = f2_pack(neg_mu, neg_mu);
+      uint64_t ls2[2] = {f2_pack(0.f, 0.f), f2_pack(0.f, 0.f)};
+#pragma unroll
+      for (int pc = 0; pc < 2; ++pc) {
+        if (pc * 32 < N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[pc][2 * i]), __uint_as_float(sr[pc][2 * i + 1])), sl2x2, nmu2),
+                      x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            ls2[i & 1] = f2_add(ls2[i & 1], f2_pack(p0, p1));
+            pk[i] = pack_bf16(p0, p1);
+          }
+          tmem_st16(tmem + 64 * b + lane_off + pc * 16, pk);
+        }
+      }
+      {
+        float a0, a1, b0, b1;
+        f2_unpack(ls2[0], a0, a1);
+        f2_unpack(ls2[1], b0, b1);
+        l += (a0 + a1) + (b0 + b1);
+      }
       if (st > 0) {
         // Observe every PV completion in order (PV(st-1) here): a parity wait
         // is only unambiguous while the barrier is at most one phase ahead.
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (st - 1) & 1, ab));
         if (!ok) break;
-      }
-      if (st > 0 && __any_sync(0xffffffffu, resc)) {
-        // O holds steps < st: rescale this warp's rows
-        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+          // O holds steps < st: rescale this warp's rows before PV(st)
+          tc_fence_after();
 #pragma unroll
-        for (int pc = 0; pc < D / 32; ++pc) {
-          uint32_t r[32];
-          tmem_ld32(tO + lane_off + pc * 32, r);
-          tmem_wait_ld();
+          for (int pc = 0; pc < D / 32; ++pc) {
+            uint32_t r[32];
+            tmem_ld32(tO + lane_off + pc * 32, r);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-          tmem_st32(tO + lane_off + pc * 32, r);
-        }
-      }
-      l *= alpha;
-      m_used = m_new;
-      const float neg_mu = (m_used == -INFINITY) ? 0.f : -m_used;
-      float lsum = 0.f;
-#pragma unroll
-      for (int pc = 0; pc < 4; ++pc) {
-        if (pc * 32 < N) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            const float p0 = ex2(fmaf(__uint_as_float(sr[pc][2 * i]), sl2, neg_mu));
-            const float p1 = ex2(fmaf(__uint_as_float(sr[pc][2 * i + 1]), sl2, neg_mu));
-            lsum += p0 + p1;
-            pk[i] = pack_bf16(p0, p1);
+            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+            tmem_st32(tO + lane_off + pc * 32, r);
           }
-          tmem_st16(tmem + 128 * b + lane_off + pc * 16, pk);
         }
       }
-      l += lsum;
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) mw[i] = mw_next[i];
+      mw[0] = mw_next[0];
+      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = mbar_wait(o_done, (n_steps - 1) & 1, ab);
@@ -301,7 +333,7 @@ __global__ void __launch_bounds__(256, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -333,7 +365,7 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
   cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   if (a.n_work == 0) return cudaSuccess;
-  fwd_kernel<D><<<static_cast<unsigned>(a.n_work), 256, C::kSmem, st>>>(
+  fwd_kernel<D><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
       tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.err);
   return cudaGetLastError();
 }
