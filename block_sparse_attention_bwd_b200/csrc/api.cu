@@ -34,19 +34,24 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [rows_per_bh, head_dim] bf16 matrices stacked over batch*heads; boxes of
-// 16 rows x 64 columns, 128-byte swizzle (the layout the MMA descriptors
-// expect).  Rows past the end of a (batch, head) read as zeros.
-bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+// `box_rows` rows x 64 columns, 128-byte swizzle (the layout the MMA
+// descriptors expect).  Rows past the end of a (batch, head) read as zeros.
+bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(head_dim) * 2 * rows};
-  cuuint32_t box[3] = {64, 16, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool make_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  return make_map(&t->m16, ptr, head_dim, rows, bh, 16) && make_map(&t->m32, ptr, head_dim, rows, bh, 32) &&
+         make_map(&t->m64, ptr, head_dim, rows, bh, 64);
 }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -93,8 +98,8 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
 }  // namespace
 
 // Entry points for other translation units of the library.
-bool make_tensor_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
-  return make_map(m, ptr, head_dim, rows, bh);
+bool make_tensor_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  return make_pages(t, ptr, head_dim, rows, bh);
 }
 TileArgs make_tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots) {
   return tile_args(P, w, own_slots, col_slots);
@@ -136,9 +141,9 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return SPATTN_ERR_INVALID_ARG;
   const int D = plan->head_dim;
   const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
-  CUtensorMap tq, tk, tv;
-  if (!make_map(&tq, q, D, plan->q.slots, bh) || !make_map(&tk, k, D, plan->k.slots, bh) ||
-      !make_map(&tv, v, D, plan->k.slots, bh))
+  TmaPages tq, tk, tv;
+  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh) ||
+      !make_pages(&tv, v, D, plan->k.slots, bh))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* O = static_cast<__nv_bfloat16*>(o);
@@ -163,9 +168,9 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
     return SPATTN_ERR_INVALID_ARG;
   const int D = plan->head_dim;
   const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_map(&tq, q, D, plan->q.slots, bh) || !make_map(&tk, k, D, plan->k.slots, bh) ||
-      !make_map(&tv, v, D, plan->k.slots, bh) || !make_map(&tdo, d_o, D, plan->q.slots, bh))
+  TmaPages tq, tk, tv, tdo;
+  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh) ||
+      !make_pages(&tv, v, D, plan->k.slots, bh) || !make_pages(&tdo, d_o, D, plan->q.slots, bh))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* dQ = static_cast<__nv_bfloat16*>(dq);
@@ -182,7 +187,7 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
     });
   if (e == cudaSuccess)
     e = timed(plan, SPATTN_K_DQ, s, [&] {
-      return launch_dq(D, tq, tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse,
+      return launch_dq(D, static_cast<const __nv_bfloat16*>(q), tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse,
                        plan->d_delta, dQ, s);
     });
   if (e == cudaSuccess && !plan->k_invalid_pages.empty())

@@ -12,9 +12,10 @@
 // softmax attention: P = exp(S - LSE), dV = P^T dO, dP = dO V^T,
 // dS = P * (dP - Delta), dK = scale dS^T Q, dQ = scale dS K.
 //
-// Both tile kernels use the CTA layout of the forward kernel: warp 0 is the
-// TMA producer, warp 1 allocates TMEM and issues tcgen05 MMAs, warps 4..7
-// own one tile row each.
+// Both tile kernels use 11 warps: warp 0 is the TMA producer, warp 1
+// allocates TMEM and issues the two products of each step, warp 10 issues
+// the accumulating product, and warps 2..9 turn each step's scores into
+// P / dS, one tile row per lane, two warp groups per step (32 columns each).
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -69,6 +70,14 @@ __global__ void delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfl
 constexpr int kBwdStepPages = 4;                  // 64 columns per step
 constexpr int kStageChunk = 64 * 128;             // one 64-column chunk of a 64-row stage
 
+// The row threads of a step split its 64 fp32 columns into two groups of 32
+// (group g reads columns [32g, 32g + 32) of the buffer).  Each group writes
+// its 16 packed bf16-pair columns back at the start of its OWN range, never
+// into the other group's, so one group's store cannot overwrite fp32 values
+// the other group has not loaded yet.  Page j of the step (16 keys = 8 pair
+// columns) therefore sits at column ds_col(j) of the buffer.
+__device__ __forceinline__ uint32_t ds_col(int j) { return static_cast<uint32_t>((j >> 1) * 32 + (j & 1) * 8); }
+
 template <int D>
 struct DkvCfg {
   static constexpr int kNch = D / 64;
@@ -80,16 +89,21 @@ struct DkvCfg {
   static constexpr int kSmem = 2 * kTile + kQStages * kStageTile + kDStages * (kStageTile + kLdBytes) + 1024 + 512;
 };
 
-// 10 warps: 0 = TMA producer, 1 = TMEM owner and MMA issuer, 2..9 = two
-// groups of row threads; group g (warps 2+4g .. 5+4g) handles columns
-// 32g .. 32g+31 of every 64-column step (warp w reaches TMEM lanes of
-// quarter w%4).
-constexpr int kBwdThreads = 320;
+// 11 warps: 0 = TMA producer, 1 = TMEM owner and issuer of the MMAs that
+// read the step's column tiles into TMEM (S^T/dP^T or S/dP), 2..9 = two
+// groups of row threads, 10 = issuer of the accumulating MMAs (dV/dK or dQ).
+// Row group g (warps 2+4g .. 5+4g) handles columns 32g .. 32g+31 of every
+// 64-column step (warp w reaches TMEM lanes of quarter w%4).  The tensor
+// core accepts only a couple of MMAs ahead of the one it runs, so a single
+// issuing warp idles it whenever that warp waits; with two issuers one keeps
+// it busy while the other waits.
+constexpr int kBwdThreads = 352;
+constexpr int kAccWarp = 10;
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    dkdv_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+    dkdv_kernel(const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
+                const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_do,
                 const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
                 const uint64_t* __restrict__ col_masks, const float* __restrict__ lse,
                 const float* __restrict__ delta, __nv_bfloat16* __restrict__ out_dk,
@@ -114,9 +128,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* st_full = ld_full + DS;  // [2]
   uint64_t* pt_full = st_full + 2;   // [2]
   uint64_t* acc_done = pt_full + 2;
-  uint64_t* acc_step = acc_done + 1;  // completes once per step's dV, dK MMAs
-  uint64_t* drain = acc_step + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* acc_b = acc_done + 1;     // [2] dV, dK MMAs of the steps using buffer b finished
+  uint64_t* drain = acc_b + 2;        // [2] one per issuing warp
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
 
@@ -128,7 +142,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(own_full, 1);
-    mbar_init(acc_step, 1);
+    mbar_init(&acc_b[0], 1);
+    mbar_init(&acc_b[1], 1);
+    mbar_init(&drain[1], 1);
     for (int s = 0; s < QS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
@@ -159,19 +175,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ahead) and issues that page's TMA boxes; every lane then fetches LSE2 and
     // Delta for two of the step's 64 query columns.
     if (lane == 0) {
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_k.m64);
+      tma_prefetch_desc(&tm_v.m64);
+      tma_prefetch_desc(&tm_q.m64);
+      tma_prefetch_desc(&tm_do.m64);
       mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
     }
     __syncwarp();
-    if (lane < wk.n_own)
-#pragma unroll
-      for (int c = 0; c < C::kNch; ++c) {
-        tma_load_3d(sK + c * kChunkBytes + lane * 2048, &tm_k, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
-        tma_load_3d(sV + c * kChunkBytes + lane * 2048, &tm_v, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
-      }
+    {
+      const int own_pid = lane < wk.n_own ? wk.own_page(lane) : 0;
+      load_page_runs<C::kNch>(sK, kChunkBytes, tm_k, own_pid, wk.n_own, wk.bh, own_full);
+      load_page_runs<C::kNch>(sV, kChunkBytes, tm_v, own_pid, wk.n_own, wk.bh, own_full);
+    }
     int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int q_issued = 0, d_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
@@ -183,19 +198,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (st >= QS && !__all_sync(0xffffffffu, mbar_wait(&q_empty[qs], ((st / QS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&q_full[qs], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sQ + qs * C::kStageTile + c * kStageChunk + lane * 2048, &tm_q, c * 64, pid * 16, wk.bh, &q_full[qs]);
+      load_page_runs<C::kNch>(sQ + qs * C::kStageTile, kStageChunk, tm_q, pid, n, wk.bh, &q_full[qs]);
       q_issued = st + 1;
       if (st >= DS && !__all_sync(0xffffffffu, mbar_wait(&do_empty[ds], ((st / DS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&do_full[ds], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sDO + ds * C::kStageTile + c * kStageChunk + lane * 2048, &tm_do, c * 64, pid * 16, wk.bh,
-                      &do_full[ds]);
+      load_page_runs<C::kNch>(sDO + ds * C::kStageTile, kStageChunk, tm_do, pid, n, wk.bh, &do_full[ds]);
       d_issued = st + 1;
       float* sl = sLD + ds * 128;
 #pragma unroll
@@ -220,40 +228,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (warp-wide; one elected lane issues) ----------------
+    // ---------------- S^T, dP^T issuer (warp-wide; one elected lane issues) ----------------
     const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
     const uint64_t dqk = sdesc_sw128(smem_u32(sQ), 16, 1024);             // Q stages, K-major
     const uint64_t ddk = sdesc_sw128(smem_u32(sDO), 16, 1024);            // dO stages, K-major
-    const uint64_t dqm = sdesc_sw128(smem_u32(sQ), kStageChunk, 1024);    // Q stages, MN-major
-    const uint64_t ddm = sdesc_sw128(smem_u32(sDO), kStageChunk, 1024);   // dO stages, MN-major
-    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
     bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
     tc_fence_after();
-    auto issue_acc = [&](int st) -> bool {
-      const int b = st & 1, qs = st % QS, ds = st % DS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (st >> 1) & 1, ab))) return false;
-      tc_fence_after();
-      const int n = min(NP, n_cols - st * NP);
-      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile), bd = sdesc_add(ddm, ds * C::kStageTile);
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n) umma_ts_w(tDV, tmem + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&do_empty[ds]);
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n)
-          umma_ts_w(tDK, tmem + 128 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&q_empty[qs]);
-      umma_commit_w(acc_step);
-      return true;
-    };
     for (int st = 0; ok && st < n_steps; ++st) {
       const int b = st & 1, qs = st % QS, ds = st % DS;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      // buffers b still feed dV(st-2) / dK(st-2) as TMEM A operands
-      bool w = (st < 2 || mbar_wait(acc_step, (st - 2) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
+      // buffers b still feed dV(st-2) / dK(st-2), issued by the other warp
+      bool w = (st < 2 || mbar_wait(&acc_b[b], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile), bd = sdesc_add(ddk, ds * C::kStageTile);
@@ -268,11 +255,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         umma_ss_w(tmem + 128 + 64 * b, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
       umma_commit_w(&st_full[b]);
-      if (st >= 1 && !issue_acc(st - 1)) ok = false;
     }
-    if (ok && n_steps > 0 && issue_acc(n_steps - 1)) umma_commit_w(acc_done);
-    umma_commit_w(drain);
-    mbar_wait_drain(drain, 0);
+    umma_commit_w(&drain[0]);
+    mbar_wait_drain(&drain[0], 0);
+  } else if (warp == kAccWarp) {
+    // ---------------- dV, dK issuer (warp-wide; one elected lane issues) ----------------
+    const uint64_t dqm = sdesc_sw128(smem_u32(sQ), kStageChunk, 1024);    // Q stages, MN-major
+    const uint64_t ddm = sdesc_sw128(smem_u32(sDO), kStageChunk, 1024);   // dO stages, MN-major
+    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
+    bool ok = true;
+    for (int st = 0; ok && st < n_steps; ++st) {
+      const int b = st & 1, qs = st % QS, ds = st % DS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (st >> 1) & 1, ab))) { ok = false; break; }
+      tc_fence_after();
+      const int n = min(NP, n_cols - st * NP);
+      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile), bd = sdesc_add(ddm, ds * C::kStageTile);
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < n) umma_ts_w(tDV, tmem + 64 * b + ds_col(j), sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&do_empty[ds]);
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < n)
+          umma_ts_w(tDK, tmem + 128 + 64 * b + ds_col(j), sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&q_empty[qs]);
+      umma_commit_w(&acc_b[b]);
+    }
+    if (ok && n_steps > 0) umma_commit_w(acc_done);
+    umma_commit_w(&drain[1]);
+    mbar_wait_drain(&drain[1], 0);
   } else {
     // ---------------- P^T, dS^T (one key row per thread) + epilogue ----------------
     const int grp = (warp - 2) >> 2;  // column half of each step
@@ -306,35 +317,67 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float4* sl4 = reinterpret_cast<const float4*>(sLD + ds * 128 + grp * 32);
         const float4* sd4 = reinterpret_cast<const float4*>(sLD + ds * 128 + 64 + grp * 32);
         uint32_t pp[16], pd[16];
+        if (m == 0xFFFFFFFFu) {
+          // every column allowed: no masking, all values finite
 #pragma unroll
-        for (int i4 = 0; i4 < 8; ++i4) {
-          const float4 L = sl4[i4];
-          const float4 Dl = sd4[i4];
-          float x0, x1, x2, x3;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
-                           f2_pack(-L.x, -L.y)), x0, x1);
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
-                           f2_pack(-L.z, -L.w)), x2, x3);
-          float p[4] = {ex2(x0), ex2(x1), ex2(x2), ex2(x3)};
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 L = sl4[i4];
+            const float4 Dl = sd4[i4];
+            float p0, p1, p2, p3, s0, s1, s2, s3;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
+                             f2_pack(-L.x, -L.y)), p0, p1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
+                             f2_pack(-L.z, -L.w)), p2, p3);
+            p0 = ex2(p0);
+            p1 = ex2(p1);
+            p2 = ex2(p2);
+            p3 = ex2(p3);
+            f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])),
+                                                      f2_pack(-Dl.x, -Dl.y))), s0, s1);
+            f2_unpack(f2_mul(f2_pack(p2, p3), f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
+                                                      f2_pack(-Dl.z, -Dl.w))), s2, s3);
+            pp[2 * i4] = pack_bf16(p0, p1);
+            pp[2 * i4 + 1] = pack_bf16(p2, p3);
+            pd[2 * i4] = pack_bf16(s0, s1);
+            pd[2 * i4 + 1] = pack_bf16(s2, s3);
+          }
+        } else if (m == 0u) {
 #pragma unroll
-          for (int h = 0; h < 4; ++h)
-            if (!((m >> (4 * i4 + h)) & 1u)) p[h] = 0.f;
-          float g0, g1, g2, g3;
-          f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])), f2_pack(-Dl.x, -Dl.y)),
-                    g0, g1);
-          f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
-                           f2_pack(-Dl.z, -Dl.w)), g2, g3);
-          float s0, s1, s2, s3;
-          f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_pack(g0, g1)), s0, s1);
-          f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_pack(g2, g3)), s2, s3);
-          pp[2 * i4] = pack_bf16(p[0], p[1]);
-          pp[2 * i4 + 1] = pack_bf16(p[2], p[3]);
-          // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
-          pd[2 * i4] = pack_bf16(p[0] != 0.f ? s0 : 0.f, p[1] != 0.f ? s1 : 0.f);
-          pd[2 * i4 + 1] = pack_bf16(p[2] != 0.f ? s2 : 0.f, p[3] != 0.f ? s3 : 0.f);
+          for (int i = 0; i < 16; ++i) {
+            pp[i] = 0u;
+            pd[i] = 0u;
+          }
+        } else {
+#pragma unroll
+          for (int i4 = 0; i4 < 8; ++i4) {
+            const float4 L = sl4[i4];
+            const float4 Dl = sd4[i4];
+            float x0, x1, x2, x3;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
+                             f2_pack(-L.x, -L.y)), x0, x1);
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
+                             f2_pack(-L.z, -L.w)), x2, x3);
+            float p[4] = {ex2(x0), ex2(x1), ex2(x2), ex2(x3)};
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              if (!((m >> (4 * i4 + h)) & 1u)) p[h] = 0.f;
+            float g0, g1, g2, g3;
+            f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])), f2_pack(-Dl.x, -Dl.y)),
+                      g0, g1);
+            f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
+                             f2_pack(-Dl.z, -Dl.w)), g2, g3);
+            float s0, s1, s2, s3;
+            f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_pack(g0, g1)), s0, s1);
+            f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_pack(g2, g3)), s2, s3);
+            pp[2 * i4] = pack_bf16(p[0], p[1]);
+            pp[2 * i4 + 1] = pack_bf16(p[2], p[3]);
+            // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
+            pd[2 * i4] = pack_bf16(p[0] != 0.f ? s0 : 0.f, p[1] != 0.f ? s1 : 0.f);
+            pd[2 * i4 + 1] = pack_bf16(p[2] != 0.f ? s2 : 0.f, p[3] != 0.f ? s3 : 0.f);
+          }
         }
-        tmem_st16(tmem + 64 * b + lane_off + grp * 16, pp);
-        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 16, pd);
+        tmem_st16(tmem + 64 * b + lane_off + grp * 32, pp);
+        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 32, pd);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -378,22 +421,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ----------------------------------------------------------------------------
 // K4: dQ (query-owned tiles, key pages as columns; the forward lists)
 // ----------------------------------------------------------------------------
-// TMEM columns: S / dS double buffer at 0 and 64, dP double buffer at 128
-// and 192, dQ at 256.  K stays in its stage until the dQ MMA of its step.
+// TMEM columns: the owned Q rows as bf16 pairs at 0 (the A operand of
+// S = Q K^T, so that MMA reads only K from shared memory), S / dS triple
+// buffer at 64, 128, 192, dP double buffer at 256, 320, dQ at 384.  With three
+// S buffers the MMA that reuses one waits for the dQ of three steps back,
+// which has long finished.
 template <int D>
 struct DqCfg {
   static constexpr int kNch = D / 64;
-  static constexpr int kTile = kNch * kChunkBytes;
-  static constexpr int kStageTile = kNch * kStageChunk;
-  static constexpr int kKStages = (D == 128) ? 5 : 8;
-  static constexpr int kVStages = (D == 128) ? 4 : 8;
-  static constexpr int kSmem = 2 * kTile + (kKStages + kVStages) * kStageTile + 1024 + 512;
+  static constexpr int kTile = kNch * kChunkBytes;        // dO tile (128 rows)
+  static constexpr int kStageTile = kNch * kStageChunk;   // 64-row K / V stage
+  static constexpr int kKStages = (D == 128) ? 6 : 10;
+  static constexpr int kVStages = (D == 128) ? 5 : 10;
+  static constexpr int kSmem = kTile + (kKStages + kVStages) * kStageTile + 1024 + 512;
 };
 
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-              const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+    dq_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ TmaPages tm_do,
+              const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
               const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
               const uint64_t* __restrict__ col_masks, const float* __restrict__ lse, const float* __restrict__ delta,
               __nv_bfloat16* __restrict__ out_dq, int64_t q_slots, float sl2, float scale, int* err) {
@@ -401,22 +447,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   constexpr int KS = C::kKStages, VS = C::kVStages, NP = kBwdStepPages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* sQ = smem;
-  uint8_t* sDO = smem + C::kTile;
-  uint8_t* sK = smem + 2 * C::kTile;       // K stage s at sK + s*kStageTile
+  uint8_t* sDO = smem;
+  uint8_t* sK = smem + C::kTile;           // K stage s at sK + s*kStageTile
   uint8_t* sV = sK + KS * C::kStageTile;   // V stage s at sV + s*kStageTile
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kStageTile);
   uint64_t* own_full = bars;
-  uint64_t* k_full = own_full + 1;
+  uint64_t* q_ready = own_full + 1;  // Q rows stored into TMEM by the row threads
+  uint64_t* k_full = q_ready + 1;
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
-  uint64_t* sd_full = v_empty + VS;  // [2]
-  uint64_t* ds_full = sd_full + 2;   // [2]
-  uint64_t* acc_done = ds_full + 2;
-  uint64_t* dq_step = acc_done + 1;  // completes once per step's dQ MMAs
-  uint64_t* drain = dq_step + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sd_full = v_empty + VS;  // [2] S and dP of a step are ready
+  uint64_t* ds_full = sd_full + 2;   // [2] dS of a step is in TMEM
+  uint64_t* dq_done = ds_full + 2;   // [3] dQ MMAs of the steps using S buffer b finished
+  uint64_t* acc_done = dq_done + 3;
+  uint64_t* drain = acc_done + 1;    // [2] one per issuing warp
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
 
@@ -428,6 +474,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(own_full, 1);
+    mbar_init(q_ready, 256);
     for (int s = 0; s < KS; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -440,9 +487,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&sd_full[b], 1);
       mbar_init(&ds_full[b], 256);
     }
+    for (int b = 0; b < 3; ++b) mbar_init(&dq_done[b], 1);
     mbar_init(acc_done, 1);
-    mbar_init(dq_step, 1);
-    mbar_init(drain, 1);
+    mbar_init(&drain[0], 1);
+    mbar_init(&drain[1], 1);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tslot, 512);
@@ -450,24 +498,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t tDQ = tmem + 256;
+  const uint32_t tQ = tmem, tDQ = tmem + 384;
+  auto tS = [&](int b3) { return tmem + 64 + 64 * b3; };
+  auto tDP = [&](int b2) { return tmem + 256 + 64 * b2; };
 
   if (warp == 0) {
     // ---------------- producer (whole warp; lane j owns page j of a step) ----------------
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_do);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
-      mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
+      tma_prefetch_desc(&tm_do.m64);
+      tma_prefetch_desc(&tm_k.m64);
+      tma_prefetch_desc(&tm_v.m64);
+      mbar_arrive_expect_tx(own_full, wk.n_own * C::kNch * 2048);
     }
     __syncwarp();
-    if (lane < wk.n_own)
-#pragma unroll
-      for (int c = 0; c < C::kNch; ++c) {
-        tma_load_3d(sQ + c * kChunkBytes + lane * 2048, &tm_q, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
-        tma_load_3d(sDO + c * kChunkBytes + lane * 2048, &tm_do, c * 64, wk.own_page(lane) * 16, wk.bh, own_full);
-      }
+    load_page_runs<C::kNch>(sDO, kChunkBytes, tm_do, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh,
+                            own_full);
     int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int k_issued = 0, v_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
@@ -479,18 +524,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sK + ks * C::kStageTile + c * kStageChunk + lane * 2048, &tm_k, c * 64, pid * 16, wk.bh, &k_full[ks]);
+      load_page_runs<C::kNch>(sK + ks * C::kStageTile, kStageChunk, tm_k, pid, n, wk.bh, &k_full[ks]);
       k_issued = st + 1;
       if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sV + vs * C::kStageTile + c * kStageChunk + lane * 2048, &tm_v, c * 64, pid * 16, wk.bh, &v_full[vs]);
+      load_page_runs<C::kNch>(sV + vs * C::kStageTile, kStageChunk, tm_v, pid, n, wk.bh, &v_full[vs]);
       v_issued = st + 1;
     }
     if (lane == 0) {
@@ -499,54 +538,58 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (warp-wide; one elected lane issues) ----------------
-    const uint64_t dq0 = sdesc_sw128(smem_u32(sQ), 16, 1024);
+    // ---------------- S, dP issuer (warp-wide; one elected lane issues) ----------------
     const uint64_t ddo0 = sdesc_sw128(smem_u32(sDO), 16, 1024);
     const uint64_t dkk = sdesc_sw128(smem_u32(sK), 16, 1024);            // K stages, K-major
-    const uint64_t dkm = sdesc_sw128(smem_u32(sK), kStageChunk, 1024);   // K stages, MN-major
     const uint64_t dvk = sdesc_sw128(smem_u32(sV), 16, 1024);            // V stages, K-major
-    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
+    bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab) && mbar_wait(q_ready, 0, ab));
     tc_fence_after();
-    auto issue_dq = [&](int st) -> bool {
-      const int b = st & 1, ks = st % KS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[b], (st >> 1) & 1, ab))) return false;
-      tc_fence_after();
-      const int n = min(NP, n_cols - st * NP);
-      const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile);
-#pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n) umma_ts_w(tDQ, tmem + 64 * b + 8 * j, sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&k_empty[ks]);
-      umma_commit_w(dq_step);
-      return true;
-    };
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b = st & 1, ks = st % KS, vs = st % VS;
+      const int b2 = st & 1, b3 = st % 3, ks = st % KS, vs = st % VS;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      // buffer b still feeds dQ(st-2) as its TMEM A operand
-      bool w = (st < 2 || mbar_wait(dq_step, (st - 2) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
+      // S buffer b3 still feeds dQ(st-3) (issued by the other warp); per-buffer
+      // barrier, waited in order
+      bool w = (st < 3 || mbar_wait(&dq_done[b3], ((st / 3) - 1) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint64_t bk = sdesc_add(dkk, ks * C::kStageTile), bv = sdesc_add(dvk, vs * C::kStageTile);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
-                  sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (st / VS) & 1, ab))) { ok = false; break; }
+        umma_ts_w(tS(b3), tQ + 8 * kk, sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      // dP buffer b2 is free once the row threads finished step st-2
+      w = (st < 2 || mbar_wait(&ds_full[b2], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&v_full[vs], (st / VS) & 1, ab);
+      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 128 + 64 * b, sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+        umma_ss_w(tDP(b2), sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bv, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
       umma_commit_w(&v_empty[vs]);
-      umma_commit_w(&sd_full[b]);
-      if (st >= 1 && !issue_dq(st - 1)) ok = false;
+      umma_commit_w(&sd_full[b2]);
     }
-    if (ok && n_steps > 0 && issue_dq(n_steps - 1)) umma_commit_w(acc_done);
-    umma_commit_w(drain);
-    mbar_wait_drain(drain, 0);
+    umma_commit_w(&drain[0]);
+    mbar_wait_drain(&drain[0], 0);
+  } else if (warp == kAccWarp) {
+    // ---------------- dQ issuer (warp-wide; one elected lane issues) ----------------
+    const uint64_t dkm = sdesc_sw128(smem_u32(sK), kStageChunk, 1024);   // K stages, MN-major
+    const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
+    bool ok = true;
+    for (int st = 0; ok && st < n_steps; ++st) {
+      const int b2 = st & 1, b3 = st % 3, ks = st % KS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[b2], (st >> 1) & 1, ab))) { ok = false; break; }
+      tc_fence_after();
+      const int n = min(NP, n_cols - st * NP);
+      const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile);
+#pragma unroll
+      for (int j = 0; j < NP; ++j)
+        if (j < n) umma_ts_w(tDQ, tS(b3) + ds_col(j), sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+      umma_commit_w(&k_empty[ks]);
+      umma_commit_w(&dq_done[b3]);
+    }
+    if (ok && n_steps > 0) umma_commit_w(acc_done);
+    umma_commit_w(&drain[1]);
+    mbar_wait_drain(&drain[1], 0);
   } else {
     const int grp = (warp - 2) >> 2;  // column half of each step
     const int q4 = warp & 3;
@@ -555,9 +598,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t code = wk.row_code(row);
     const int seg = code < 4 ? static_cast<int>(code) : -1;
     const bool owned = code != 15u && row < 16 * wk.n_own;
-    const int64_t slot = owned ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+    const int64_t slot = row < 16 * wk.n_own ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+    const bool loaded = row < 16 * wk.n_own && slot < q_slots;
     const bool valid_slot = owned && slot < q_slots;
     const int64_t roff = static_cast<int64_t>(wk.bh) * q_slots + slot;
+    // Q row into TMEM as bf16 pairs: group g stores pair columns [g*D/4, (g+1)*D/4)
+    {
+      constexpr int kCols = D / 4;  // 32-bit TMEM columns per group
+      uint32_t qr[32] = {};
+      if (loaded) {
+        const uint4* src = reinterpret_cast<const uint4*>(q + roff * D + grp * (D / 2));
+#pragma unroll
+        for (int i = 0; i < kCols / 4; ++i) {
+          const uint4 v = __ldg(src + i);
+          qr[4 * i] = v.x;
+          qr[4 * i + 1] = v.y;
+          qr[4 * i + 2] = v.z;
+          qr[4 * i + 3] = v.w;
+        }
+      }
+      if (kCols == 32) {
+        tmem_st32(tQ + lane_off + grp * kCols, qr);
+      } else {
+        uint32_t h[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) h[i] = qr[i];
+        tmem_st16(tQ + lane_off + grp * kCols, h);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(q_ready);
+    }
     const float lse2 = (valid_slot && seg >= 0) ? __ldg(lse + roff) * kLog2e : 0.f;
     const float dl = (valid_slot && seg >= 0) ? __ldg(delta + roff) : 0.f;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -567,16 +638,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t mw[2];
     if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
-      const int b = st & 1;
+      const int b2 = st & 1, b3 = st % 3;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b2], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
       uint32_t a[32], d[32];
       if (active) {
-        tmem_ld32(tmem + 64 * b + lane_off + grp * 32, a);
-        tmem_ld32(tmem + 128 + 64 * b + lane_off + grp * 32, d);
+        tmem_ld32(tS(b3) + lane_off + grp * 32, a);
+        tmem_ld32(tDP(b2) + lane_off + grp * 32, d);
       }
       uint32_t mw_next[2] = {0u, 0u};
       if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
@@ -584,23 +655,39 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_wait_ld();
         const uint32_t m = grp ? mw[1] : mw[0];
         uint32_t pd[16];
+        if (m == 0xFFFFFFFFu) {
+          // every column allowed: no masking, all values finite
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2, nl2), x0, x1);
-          float p0 = ex2(x0), p1 = ex2(x1);
-          if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
-          if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
-          float g0, g1;
-          f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), ndl)),
-                    g0, g1);
-          pd[i] = pack_bf16(p0 != 0.f ? g0 : 0.f, p1 != 0.f ? g1 : 0.f);
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1, g0, g1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2, nl2), x0, x1);
+            f2_unpack(f2_mul(f2_pack(ex2(x0), ex2(x1)),
+                             f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), ndl)),
+                      g0, g1);
+            pd[i] = pack_bf16(g0, g1);
+          }
+        } else if (m == 0u) {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) pd[i] = 0u;
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2, nl2), x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
+            if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
+            float g0, g1;
+            f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1])), ndl)),
+                      g0, g1);
+            pd[i] = pack_bf16(p0 != 0.f ? g0 : 0.f, p1 != 0.f ? g1 : 0.f);
+          }
         }
-        tmem_st16(tmem + 64 * b + lane_off + grp * 16, pd);
+        tmem_st16(tS(b3) + lane_off + grp * 32, pd);
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&ds_full[b]);
+      mbar_arrive(&ds_full[b2]);
       mw[0] = mw_next[0];
       mw[1] = mw_next[1];
     }
@@ -647,8 +734,8 @@ cudaError_t launch_delta(int head_dim, const __nv_bfloat16* o, const __nv_bfloat
 }
 
 template <int D>
-static cudaError_t launch_dkdv_t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                                 const CUtensorMap& tdo, const TileArgs& a, const float* lse, const float* delta,
+static cudaError_t launch_dkdv_t(const TmaPages& tk, const TmaPages& tv, const TmaPages& tq,
+                                 const TmaPages& tdo, const TileArgs& a, const float* lse, const float* delta,
                                  __nv_bfloat16* dk, __nv_bfloat16* dv, cudaStream_t st) {
   using C = DkvCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -660,29 +747,29 @@ static cudaError_t launch_dkdv_t(const CUtensorMap& tk, const CUtensorMap& tv, c
 }
 
 template <int D>
-static cudaError_t launch_dq_t(const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                               const CUtensorMap& tv, const TileArgs& a, const float* lse, const float* delta,
+static cudaError_t launch_dq_t(const __nv_bfloat16* q, const TmaPages& tdo, const TmaPages& tk,
+                               const TmaPages& tv, const TileArgs& a, const float* lse, const float* delta,
                                __nv_bfloat16* dq, cudaStream_t st) {
   using C = DqCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
   dq_kernel<D><<<static_cast<unsigned>(a.n_work), kBwdThreads, C::kSmem, st>>>(
-      tq, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.err);
+      q, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.err);
   return cudaGetLastError();
 }
 
-cudaError_t launch_dkdv(int head_dim, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                        const CUtensorMap& tdo, const TileArgs& a, const float* lse, const float* delta,
-                        __nv_bfloat16* dk, __nv_bfloat16* dv, cudaStream_t st) {
+cudaError_t launch_dkdv(int head_dim, const TmaPages& tk, const TmaPages& tv, const TmaPages& tq, const TmaPages& tdo,
+                        const TileArgs& a, const float* lse, const float* delta, __nv_bfloat16* dk,
+                        __nv_bfloat16* dv, cudaStream_t st) {
   return head_dim == 128 ? launch_dkdv_t<128>(tk, tv, tq, tdo, a, lse, delta, dk, dv, st)
                          : launch_dkdv_t<64>(tk, tv, tq, tdo, a, lse, delta, dk, dv, st);
 }
 
-cudaError_t launch_dq(int head_dim, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                      const CUtensorMap& tv, const TileArgs& a, const float* lse, const float* delta,
+cudaError_t launch_dq(int head_dim, const __nv_bfloat16* q, const TmaPages& tdo, const TmaPages& tk,
+                      const TmaPages& tv, const TileArgs& a, const float* lse, const float* delta,
                       __nv_bfloat16* dq, cudaStream_t st) {
-  return head_dim == 128 ? launch_dq_t<128>(tq, tdo, tk, tv, a, lse, delta, dq, st)
-                         : launch_dq_t<64>(tq, tdo, tk, tv, a, lse, delta, dq, st);
+  return head_dim == 128 ? launch_dq_t<128>(q, tdo, tk, tv, a, lse, delta, dq, st)
+                         : launch_dq_t<64>(q, tdo, tk, tv, a, lse, delta, dq, st);
 }
 
 }  // namespace spattn

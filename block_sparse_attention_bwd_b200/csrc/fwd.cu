@@ -52,8 +52,8 @@ constexpr int kFwdThreads = 192;
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 2)
-    fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-               const __grid_constant__ CUtensorMap tm_v, const int32_t* __restrict__ work,
+    fwd_kernel(const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_k,
+               const __grid_constant__ TmaPages tm_v, const int32_t* __restrict__ work,
                const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
                __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
                int* err) {
@@ -114,16 +114,15 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     // Lane j < n owns page j of a step: it holds the page id (fetched one step
     // ahead) and issues that page's TMA boxes.
     if (lane == 0) {
-      tma_prefetch_desc(&tm_q);
-      tma_prefetch_desc(&tm_k);
-      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_q.m64);
+      tma_prefetch_desc(&tm_k.m64);
+      tma_prefetch_desc(&tm_v.m64);
+      tma_prefetch_desc(&tm_k.m16);
+      tma_prefetch_desc(&tm_v.m16);
       mbar_arrive_expect_tx(q_full, wk.n_own * C::kNch * 2048);
     }
     __syncwarp();
-    if (lane < wk.n_own)
-#pragma unroll
-      for (int c = 0; c < C::kNch; ++c)
-        tma_load_3d(sQ + c * kChunkBytes + lane * 2048, &tm_q, c * 64, wk.own_page(lane) * 16, wk.bh, q_full);
+    load_page_runs<C::kNch>(sQ, kChunkBytes, tm_q, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh, q_full);
     int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int k_issued = 0, v_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
@@ -135,18 +134,12 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sK + ks * C::kStage + c * kFwdStageChunk + lane * 2048, &tm_k, c * 64, pid * 16, wk.bh, &k_full[ks]);
+      load_page_runs<C::kNch>(sK + ks * C::kStage, kFwdStageChunk, tm_k, pid, n, wk.bh, &k_full[ks]);
       k_issued = st + 1;
       if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
       __syncwarp();
-      if (lane < n)
-#pragma unroll
-        for (int c = 0; c < C::kNch; ++c)
-          tma_load_3d(sV + vs * C::kStage + c * kFwdStageChunk + lane * 2048, &tm_v, c * 64, pid * 16, wk.bh, &v_full[vs]);
+      load_page_runs<C::kNch>(sV + vs * C::kStage, kFwdStageChunk, tm_v, pid, n, wk.bh, &v_full[vs]);
       v_issued = st + 1;
     }
     // no copy may still be landing in shared memory when the CTA exits
@@ -261,14 +254,19 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       for (int pc = 0; pc < 2; ++pc) {
         if (pc * 32 < N) {
           uint32_t pk[16];
+          if (mw[pc] == 0u) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[pc][2 * i]), __uint_as_float(sr[pc][2 * i + 1])), sl2x2, nmu2),
-                      x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            ls2[i & 1] = f2_add(ls2[i & 1], f2_pack(p0, p1));
-            pk[i] = pack_bf16(p0, p1);
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[pc][2 * i]), __uint_as_float(sr[pc][2 * i + 1])), sl2x2, nmu2),
+                        x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              ls2[i & 1] = f2_add(ls2[i & 1], f2_pack(p0, p1));
+              pk[i] = pack_bf16(p0, p1);
+            }
           }
           tmem_st16(tmem + 64 * b + lane_off + pc * 16, pk);
         }
@@ -359,7 +357,7 @@ __global__ void fill_kernel(const int32_t* __restrict__ pages, int64_t n_bh, int
 }
 
 template <int D>
-cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const TileArgs& a,
+cudaError_t launch_fwd_t(const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
                          __nv_bfloat16* o, float* lse, cudaStream_t st) {
   using C = FwdCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
@@ -372,8 +370,8 @@ cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUt
 
 }  // namespace
 
-cudaError_t launch_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const TileArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t st) {
+cudaError_t launch_fwd(int head_dim, const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
+                       __nv_bfloat16* o, float* lse, cudaStream_t st) {
   return head_dim == 128 ? launch_fwd_t<128>(tq, tk, tv, a, o, lse, st) : launch_fwd_t<64>(tq, tk, tv, a, o, lse, st);
 }
 

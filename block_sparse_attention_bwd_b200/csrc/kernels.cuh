@@ -8,6 +8,15 @@
 
 namespace spattn {
 
+// Three TMA descriptors over the same [rows, head_dim] x (batch*heads) bf16
+// tensor, with boxes of 16, 32 and 64 rows (64 columns, 128-byte swizzle).
+// A run of consecutive 16-row pages is fetched with the fewest boxes: the TMA
+// engine's cost is per request, so one 64-row box moves 4x the bytes of a
+// page-sized box in about the same time.
+struct TmaPages {
+  CUtensorMap m16, m32, m64;
+};
+
 // Everything one attention launch needs besides its tensor maps.
 struct TileArgs {
   const int32_t* work = nullptr;    // n_work x 32 words (see spattn_plan_work)
@@ -21,21 +30,21 @@ struct TileArgs {
 };
 
 // K1: O, LSE for every query-owned work item.
-cudaError_t launch_fwd(int head_dim, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const TileArgs& a, __nv_bfloat16* o, float* lse, cudaStream_t st);
+cudaError_t launch_fwd(int head_dim, const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
+                       __nv_bfloat16* o, float* lse, cudaStream_t st);
 
 // K2: delta[row] = sum_d dO[row, d] * O[row, d] over rows = batch*heads*q_slots.
 cudaError_t launch_delta(int head_dim, const __nv_bfloat16* o, const __nv_bfloat16* d_o, float* delta,
                          int64_t rows, cudaStream_t st);
 
 // K3: dK, dV for every key-owned work item.
-cudaError_t launch_dkdv(int head_dim, const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tq,
-                        const CUtensorMap& tdo, const TileArgs& a, const float* lse, const float* delta,
-                        __nv_bfloat16* dk, __nv_bfloat16* dv, cudaStream_t st);
+cudaError_t launch_dkdv(int head_dim, const TmaPages& tk, const TmaPages& tv, const TmaPages& tq, const TmaPages& tdo,
+                        const TileArgs& a, const float* lse, const float* delta, __nv_bfloat16* dk,
+                        __nv_bfloat16* dv, cudaStream_t st);
 
-// K4: dQ for every query-owned work item.
-cudaError_t launch_dq(int head_dim, const CUtensorMap& tq, const CUtensorMap& tdo, const CUtensorMap& tk,
-                      const CUtensorMap& tv, const TileArgs& a, const float* lse, const float* delta,
+// K4: dQ for every query-owned work item (Q rows are read directly into TMEM).
+cudaError_t launch_dq(int head_dim, const __nv_bfloat16* q, const TmaPages& tdo, const TmaPages& tk,
+                      const TmaPages& tv, const TileArgs& a, const float* lse, const float* delta,
                       __nv_bfloat16* dq, cudaStream_t st);
 
 // K5: zero the rows of pages that hold no valid slot (and LSE = -inf).

@@ -51,7 +51,7 @@ int scratch_address(int dev, float** out) {
 }  // namespace
 
 // Shared with api.cu: tensor maps and tile arguments.
-bool make_tensor_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh);
+bool make_tensor_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh);
 TileArgs make_tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots);
 
 }  // namespace spattn
@@ -75,9 +75,9 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
   int st = scratch_address(dev, &delta);
   if (st) return st;
   const int D = plan->head_dim;
-  CUtensorMap tq, tk, tv, tdo;
-  if (!make_tensor_map(&tq, q, D, plan->q.slots, bh) || !make_tensor_map(&tk, k, D, plan->k.slots, bh) ||
-      !make_tensor_map(&tv, v, D, plan->k.slots, bh) || !make_tensor_map(&tdo, d_o, D, plan->q.slots, bh))
+  TmaPages tq, tk, tv, tdo;
+  if (!make_tensor_pages(&tq, q, D, plan->q.slots, bh) || !make_tensor_pages(&tk, k, D, plan->k.slots, bh) ||
+      !make_tensor_pages(&tv, v, D, plan->k.slots, bh) || !make_tensor_pages(&tdo, d_o, D, plan->q.slots, bh))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* dQ = static_cast<__nv_bfloat16*>(dq);
@@ -91,7 +91,7 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
     e = launch_dkdv(D, tk, tv, tq, tdo, make_tile_args(plan, plan->wk, plan->k.slots, plan->q.slots), lse, delta, dK,
                     dV, s);
   if (e == cudaSuccess)
-    e = launch_dq(D, tq, tdo, tk, tv, make_tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, delta, dQ, s);
+    e = launch_dq(D, static_cast<const __nv_bfloat16*>(q), tdo, tk, tv, make_tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, delta, dQ, s);
   if (e == cudaSuccess && !plan->k_invalid_pages.empty())
     e = launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots, dK,
                     dV, nullptr, s);

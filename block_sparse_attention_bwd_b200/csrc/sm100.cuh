@@ -34,21 +34,10 @@ enum : int {
   kErrBadWork = 2,   // a work item failed its device-side sanity check
 };
 
-// Deadline of one wait, in nanoseconds of %globaltimer.
-#ifndef SPATTN_WAIT_NS
-#define SPATTN_WAIT_NS 2000000000ull
-#endif
-
 struct Abort {
   volatile int* flag;     // shared-memory CTA abort flag
   int* err;               // global error word (may be null)
 };
-
-__device__ __forceinline__ uint64_t globaltimer() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -91,16 +80,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Deadline of one wait in SM clock cycles (about 2 s at 2 GHz).
+#ifndef SPATTN_WAIT_CYCLES
+#define SPATTN_WAIT_CYCLES 4000000000ll
+#endif
+
 // Wait for the phase with the given parity to complete.  Returns false if the
 // CTA is aborting or the deadline passed (then the abort flag is raised).
+// The fast path is a bare try_wait; the deadline is checked on the cheap SM
+// cycle counter once every 1024 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer();
+  long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
+    if ((it & 1023u) == 0u) {
       if (*ab.flag) return false;
-      if (globaltimer() - t0 > SPATTN_WAIT_NS) {
+      const long long now = clock64();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > SPATTN_WAIT_CYCLES) {
         raise_abort(ab, kErrTimeout);
         return false;
       }
@@ -111,10 +110,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 // Same, ignoring the abort flag (used during teardown to drain async work),
 // with a short deadline.
 __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  uint64_t t0 = globaltimer();
+  long long t0 = 0;
   for (uint32_t it = 0;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u && globaltimer() - t0 > 200000000ull) return false;
+    if ((it & 1023u) == 0u) {
+      const long long now = clock64();
+      if (t0 == 0) t0 = now;
+      else if (now - t0 > 400000000ll) return false;
+    }
   }
 }
 
@@ -263,7 +266,11 @@ __device__ __forceinline__ uint64_t sdesc_add(uint64_t desc, uint32_t bytes) {
 // ----------------------------------------------------------------------------
 // tcgen05: TMEM <-> registers (warp-collective, 32 lanes x N columns)
 // ----------------------------------------------------------------------------
+// These are .sync.aligned: all 32 lanes must execute the same instance.  Each
+// wrapper first reconverges the warp, since callers may reach it right after
+// lane-divergent code (the compiler does not guarantee reconvergence there).
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
@@ -277,6 +284,7 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
@@ -286,6 +294,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  __syncwarp();
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
       "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
@@ -297,8 +306,14 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  __syncwarp();
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
 
 // ----------------------------------------------------------------------------
 // small math helpers

@@ -2,6 +2,7 @@
 // per-row masks of one 128-column step, smem layout constants.
 #pragma once
 
+#include "kernels.cuh"
 #include "sm100.cuh"
 
 namespace spattn {
@@ -54,16 +55,36 @@ __device__ __forceinline__ void step_masks(const uint64_t* __restrict__ masks, i
   }
 }
 
-// TMA-load n 16-row pages (all 64-column chunks) into a stage whose chunks
-// are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every chunk.
+// Warp-collective TMA gather of n (<= 32) pages into a stage whose 64-column
+// chunks are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every
+// chunk.  Lane j < n holds page id `pid` of page j.  Maximal runs of
+// consecutive page ids are fetched with 64-, 32- and 16-row boxes by the
+// run's first lane.  All 32 lanes must call this.
 template <int NCH>
-__device__ __forceinline__ void load_pages(uint8_t* dst, int chunk_bytes, const CUtensorMap* map,
-                                           const int32_t* __restrict__ pages, int n, int bh, uint64_t* bar) {
-  for (int j = 0; j < n; ++j) {
-    const int row = __ldg(pages + j) * 16;
+__device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, const TmaPages& maps, int pid, int n,
+                                               int bh, uint64_t* bar) {
+  const int lane = lane_id();
+  const int nxt = __shfl_down_sync(0xffffffffu, pid, 1);
+  const unsigned cont = __ballot_sync(0xffffffffu, lane + 1 < n && nxt == pid + 1);  // bit j: page j+1 follows j
+  const bool start = lane < n && (lane == 0 || !((cont >> (lane - 1)) & 1u));
+  if (!start) return;
+  int rem = __ffs(~(cont >> lane));  // run length
+  int j = lane;
+  auto box = [&](const CUtensorMap* m, int rows) {
 #pragma unroll
-    for (int c = 0; c < NCH; ++c) tma_load_3d(dst + c * chunk_bytes + j * 2048, map, c * 64, row, bh, bar);
+    for (int c = 0; c < NCH; ++c)
+      tma_load_3d(dst + c * chunk_bytes + j * 2048, m, c * 64, (pid + (j - lane)) * 16, bh, bar);
+    j += rows / 16;
+  };
+  while (rem >= 4) {
+    box(&maps.m64, 64);
+    rem -= 4;
   }
+  if (rem >= 2) {
+    box(&maps.m32, 32);
+    rem -= 2;
+  }
+  if (rem == 1) box(&maps.m16, 16);
 }
 
 __device__ __forceinline__ float lg2(float x) {
