@@ -64,19 +64,39 @@ __global__ void delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfl
 // ----------------------------------------------------------------------------
 // K3: dK, dV (key-owned tiles, query pages as columns, 64 columns per step)
 // ----------------------------------------------------------------------------
-// TMEM columns: S^T / P^T double buffer at 0 and 64, dP^T / dS^T double
-// buffer at 128 and 192, dV at 256, dK at 256 + D.  The MMAs of step c+1
-// (S^T, dP^T) run while the row threads turn step c into P^T and dS^T.
+// TMEM columns: one fp32 staging set (S^T at 0, dP^T at 64), two packed
+// bf16 operand sets (P^T at 128 + 64p, dS^T at 160 + 64p), dV at 256, dK at
+// 256 + D.  The staging set is free again as soon as the row threads have
+// loaded it, so the S^T / dP^T MMAs of step c+1 run while the row threads
+// compute step c; the packed set of step c is reused two steps later, after
+// the dV / dK MMAs that read it.
+//
+// The per-column terms of the backward pass are folded into the two MMAs
+// with one extra K = 16 slice each, so the row threads read nothing but
+// TMEM: with x = LSE / scale of query column c, split into three bf16 terms
+// x = h + m + l (exact to about 2^-27 relative),
+//   [K | 1 1 1 0..] . [Q | -h -m -l 0..]^T = S^T - x,  sl2 * (S^T - x) = log2 P^T,
+//   [V | 1 1 1 0..] . [dO | -Delta split]^T = dP^T - Delta,
+// both accumulated in fp32.  The slices are 16 bf16 wide, in the plain
+// (unswizzled) K-major layout: a 128-row block of ones shared by both MMAs,
+// and one 64-row block per Q / dO stage that the producer writes.
 constexpr int kBwdStepPages = 4;                  // 64 columns per step
 constexpr int kStageChunk = 64 * 128;             // one 64-column chunk of a 64-row stage
+constexpr int kAugStage = 64 * 32;                // 64 rows x 16 bf16, plain layout
+constexpr int kOnesBytes = 128 * 32;              // 128 rows x 16 bf16, plain layout
 
-// The row threads of a step split its 64 fp32 columns into two groups of 32
-// (group g reads columns [32g, 32g + 32) of the buffer).  Each group writes
-// its 16 packed bf16-pair columns back at the start of its OWN range, never
-// into the other group's, so one group's store cannot overwrite fp32 values
-// the other group has not loaded yet.  Page j of the step (16 keys = 8 pair
-// columns) therefore sits at column ds_col(j) of the buffer.
-__device__ __forceinline__ uint32_t ds_col(int j) { return static_cast<uint32_t>((j >> 1) * 32 + (j & 1) * 8); }
+// Byte offset of row r (first 8 of its 16 elements) in a plain K-major
+// 16-wide block: 8-row core matrices of 256 bytes, the second K half 128 B on.
+__device__ __forceinline__ uint32_t aug_row_off(int r) { return static_cast<uint32_t>((r >> 3) * 256 + (r & 7) * 16); }
+
+// First 8 elements of an augmented row: -x as three bf16 terms, then zeros.
+__device__ __forceinline__ uint4 aug_row(float x) {
+  const float h = __bfloat162float(__float2bfloat16_rn(x));
+  const float r1 = x - h;
+  const float m = __bfloat162float(__float2bfloat16_rn(r1));
+  const float l = r1 - m;
+  return make_uint4(pack_bf16(-h, -m), pack_bf16(-l, 0.f), 0u, 0u);
+}
 
 template <int D>
 struct DkvCfg {
@@ -85,8 +105,7 @@ struct DkvCfg {
   static constexpr int kStageTile = kNch * kStageChunk;  // 64-row column stage
   static constexpr int kQStages = (D == 128) ? 4 : 6;
   static constexpr int kDStages = (D == 128) ? 4 : 6;
-  static constexpr int kLdBytes = 2 * 64 * 4;          // LSE2 and Delta of 64 columns
-  static constexpr int kSmem = 2 * kTile + kQStages * kStageTile + kDStages * (kStageTile + kLdBytes) + 1024 + 512;
+  static constexpr int kSmem = 2 * kTile + (kQStages + kDStages) * (kStageTile + kAugStage) + kOnesBytes + 1024 + 512;
 };
 
 // 11 warps: 0 = TMA producer, 1 = TMEM owner and issuer of the MMAs that
@@ -99,9 +118,14 @@ struct DkvCfg {
 // it busy while the other waits.
 constexpr int kBwdThreads = 352;
 constexpr int kAccWarp = 10;
+// dK / dV add warp 11, the producer of the dO stages (warp 0 produces the Q
+// stages): a TMA request holds its issuing thread for hundreds of cycles, so
+// one producer for both column tensors would set the step time.
+constexpr int kDkvThreads = 384;
+constexpr int kDoWarp = 11;
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     dkdv_kernel(const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
                 const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_do,
                 const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
@@ -117,18 +141,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint8_t* sV = smem + C::kTile;
   uint8_t* sQ = smem + 2 * C::kTile;                 // Q stage s at sQ + s*kStageTile
   uint8_t* sDO = sQ + QS * C::kStageTile;            // dO stage s at sDO + s*kStageTile
-  float* sLD = reinterpret_cast<float*>(sDO + DS * C::kStageTile);  // stage s: LSE2[64], Delta[64]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sLD) + DS * C::kLdBytes);
+  uint8_t* sQa = sDO + DS * C::kStageTile;           // -LSE/scale slice of Q stage s at sQa + s*kAugStage
+  uint8_t* sDa = sQa + QS * kAugStage;               // -Delta slice of dO stage s at sDa + s*kAugStage
+  uint8_t* sOnes = sDa + DS * kAugStage;             // ones slice of the owned K / V rows
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + kOnesBytes);
   uint64_t* own_full = bars;
   uint64_t* q_full = own_full + 1;
   uint64_t* q_empty = q_full + QS;
   uint64_t* do_full = q_empty + QS;
   uint64_t* do_empty = do_full + DS;
-  uint64_t* ld_full = do_empty + DS;
-  uint64_t* st_full = ld_full + DS;  // [2]
-  uint64_t* pt_full = st_full + 2;   // [2]
+  uint64_t* st_full = do_empty + DS;  // S^T, dP^T of a step are in the staging set
+  uint64_t* st_free = st_full + 1;    // the row threads have loaded the staging set
+  uint64_t* pt_full = st_free + 1;    // [2] P^T, dS^T of a step are in packed set p
   uint64_t* acc_done = pt_full + 2;
-  uint64_t* acc_b = acc_done + 1;     // [2] dV, dK MMAs of the steps using buffer b finished
+  uint64_t* acc_b = acc_done + 1;     // [2] dV, dK MMAs of the steps using packed set p finished
   uint64_t* drain = acc_b + 2;        // [2] one per issuing warp
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -152,15 +178,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < DS; ++s) {
       mbar_init(&do_full[s], 1);
       mbar_init(&do_empty[s], 1);
-      mbar_init(&ld_full[s], 32);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&st_full[b], 1);
-      mbar_init(&pt_full[b], 256);
-    }
+    mbar_init(st_full, 1);
+    mbar_init(st_free, 256);
+    for (int b = 0; b < 2; ++b) mbar_init(&pt_full[b], 256);
     mbar_init(acc_done, 1);
     mbar_init(drain, 1);
     fence_barrier_init();
+  }
+  {
+    // Slices: the ones block holds 1 1 1 0.. in every row; the Q / dO slices
+    // start at zero (their second K half is never written again).
+    uint4* sl = reinterpret_cast<uint4*>(sQa);
+    constexpr int kN16 = ((QS + DS) * kAugStage + kOnesBytes) / 16;
+    constexpr int kOnes0 = (QS + DS) * kAugStage / 16;
+    for (int i = threadIdx.x; i < kN16; i += kDkvThreads) {
+      const bool one = i >= kOnes0 && ((i - kOnes0) & 15) < 8;  // first K half of a ones row
+      sl[i] = one ? make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
   }
   if (warp == 1) tmem_alloc(tslot, 512);
   tc_fence_before();
@@ -169,63 +205,97 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   const uint32_t tmem = *tslot;
   const uint32_t tDV = tmem + 256, tDK = tmem + 256 + D;
 
-  if (warp == 0) {
-    // ---------------- producer (whole warp) ----------------
+  if (warp == 0 || warp == kDoWarp) {
+    // ---------------- producers (whole warps): warp 0 = Q stages, warp 11 = dO stages ----------------
     // Lane j < n owns page j of a step: it holds the page id (fetched one step
-    // ahead) and issues that page's TMA boxes; every lane then fetches LSE2 and
-    // Delta for two of the step's 64 query columns.
-    if (lane == 0) {
-      tma_prefetch_desc(&tm_k.m64);
-      tma_prefetch_desc(&tm_v.m64);
-      tma_prefetch_desc(&tm_q.m64);
-      tma_prefetch_desc(&tm_do.m64);
-      mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
-    }
-    __syncwarp();
-    {
+    // ahead) and issues that page's TMA boxes; every lane also writes the
+    // augmented slice rows of two of the step's 64 query columns.
+    const bool is_q = warp == 0;
+    const int NS = is_q ? QS : DS;
+    uint8_t* stage0 = is_q ? sQ : sDO;
+    uint8_t* aug0 = is_q ? sQa : sDa;
+    uint64_t* full = is_q ? q_full : do_full;
+    uint64_t* empty = is_q ? q_empty : do_empty;
+    const TmaPages& tm = is_q ? tm_q : tm_do;
+    const float* terms = is_q ? lse : delta;
+    if (is_q) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_k.m64);
+        tma_prefetch_desc(&tm_v.m64);
+        mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
+      }
+      __syncwarp();
       const int own_pid = lane < wk.n_own ? wk.own_page(lane) : 0;
       load_page_runs<C::kNch>(sK, kChunkBytes, tm_k, own_pid, wk.n_own, wk.bh, own_full);
       load_page_runs<C::kNch>(sV, kChunkBytes, tm_v, own_pid, wk.n_own, wk.bh, own_full);
     }
-    int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
-    int q_issued = 0, d_issued = 0;
-    for (int st = 0; st < n_steps; ++st) {
-      const int qs = st % QS, ds = st % DS;
-      const int n = min(NP, n_cols - st * NP);
-      const int pid = pid_next;
-      if (st + 1 < n_steps)
-        pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
-      if (st >= QS && !__all_sync(0xffffffffu, mbar_wait(&q_empty[qs], ((st / QS) - 1) & 1, ab))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&q_full[qs], n * C::kNch * 2048);
-      __syncwarp();
-      load_page_runs<C::kNch>(sQ + qs * C::kStageTile, kStageChunk, tm_q, pid, n, wk.bh, &q_full[qs]);
-      q_issued = st + 1;
-      if (st >= DS && !__all_sync(0xffffffffu, mbar_wait(&do_empty[ds], ((st / DS) - 1) & 1, ab))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&do_full[ds], n * C::kNch * 2048);
-      __syncwarp();
-      load_page_runs<C::kNch>(sDO + ds * C::kStageTile, kStageChunk, tm_do, pid, n, wk.bh, &do_full[ds]);
-      d_issued = st + 1;
-      float* sl = sLD + ds * 128;
+    if (lane == 0) {
+      tma_prefetch_desc(&tm.m64w);
+      tma_prefetch_desc(&tm.m64);
+    }
+    // Lane j holds the page id of column page j of steps st and st+1, and the
+    // per-column term (LSE for Q, Delta for dO) of columns lane and lane+32 of
+    // step st.  Both are fetched one step ahead, and the fetched values are
+    // used only in the next iteration, so their global-load latency overlaps
+    // the waits and TMA issue of the current one instead of stalling it.
+    const float inv_scale = 1.0f / scale;
+    auto page_id = [&](int s) {
+      return (s < n_steps && lane < min(NP, n_cols - s * NP)) ? __ldg(col_pages + wk.e0 + s * NP + lane) : 0;
+    };
+    // Raw loads only (nothing here reads the loaded registers); a dead column
+    // (beyond the step or the tensor) loads a valid address and is zeroed
+    // where the value is used, through its bit in `live`.
+    auto fetch_terms = [&](int s, int pg_lane, float (&x)[2], uint32_t& live) {
+      const int n_s = min(NP, n_cols - s * NP);
+      live = 0u;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int idx = lane + 32 * h;                     // column of the step
-        const int pg = __shfl_sync(0xffffffffu, pid, idx >> 4);
+        const int idx = lane + 32 * h;  // column of the step
+        const int pg = __shfl_sync(0xffffffffu, pg_lane, idx >> 4);
         const int64_t slot = static_cast<int64_t>(pg) * 16 + (idx & 15);
-        float l2 = 0.f, dl = 0.f;
-        if ((idx >> 4) < n && slot < q_slots) {
-          const int64_t off = static_cast<int64_t>(wk.bh) * q_slots + slot;
-          l2 = __ldg(lse + off) * kLog2e;
-          dl = __ldg(delta + off);
-        }
-        sl[idx] = l2;
-        sl[64 + idx] = dl;
+        const bool ok = s < n_steps && (idx >> 4) < n_s && slot < q_slots;
+        x[h] = __ldg(terms + static_cast<int64_t>(wk.bh) * q_slots + (ok ? slot : 0));
+        live |= ok ? (1u << h) : 0u;
       }
-      mbar_arrive(&ld_full[ds]);
+    };
+    // Augmented row of a column: -LSE / scale for Q (a column that attends
+    // nothing, LSE = -inf, is masked everywhere, like a dead one: zeros), or
+    // -Delta for dO.
+    auto term_row = [&](float t, bool ok) {
+      const float x = is_q ? t * inv_scale : t;
+      return aug_row(ok && isfinite(x) ? x : 0.f);
+    };
+    int pid = page_id(0), pid_next = page_id(1);
+    float xc[2];
+    uint32_t livec;
+    fetch_terms(0, pid, xc, livec);
+    int issued = 0;
+    for (int st = 0; st < n_steps; ++st) {
+      const int s = st % NS;
+      const int n = min(NP, n_cols - st * NP);
+      const int pid_next2 = page_id(st + 2);
+      float xn[2];
+      uint32_t liven;
+      fetch_terms(st + 1, pid_next, xn, liven);
+      if (st >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / NS) - 1) & 1, ab))) break;
+#pragma unroll
+      for (int h = 0; h < 2; ++h)
+        *reinterpret_cast<uint4*>(aug0 + s * kAugStage + aug_row_off(lane + 32 * h)) = term_row(xc[h], (livec >> h) & 1u);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
+      __syncwarp();
+      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
+      issued = st + 1;
+      pid = pid_next;
+      pid_next = pid_next2;
+      livec = liven;
+      xc[0] = xn[0];
+      xc[1] = xn[1];
     }
     if (lane == 0) {
-      for (int st = max(0, q_issued - QS); st < q_issued; ++st) mbar_wait_drain(&q_full[st % QS], (st / QS) & 1);
-      for (int st = max(0, d_issued - DS); st < d_issued; ++st) mbar_wait_drain(&do_full[st % DS], (st / DS) & 1);
-      mbar_wait_drain(own_full, 0);
+      for (int st = max(0, issued - NS); st < issued; ++st) mbar_wait_drain(&full[st % NS], (st / NS) & 1);
+      if (is_q) mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
     // ---------------- S^T, dP^T issuer (warp-wide; one elected lane issues) ----------------
@@ -233,28 +303,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), 16, 1024);
     const uint64_t dqk = sdesc_sw128(smem_u32(sQ), 16, 1024);             // Q stages, K-major
     const uint64_t ddk = sdesc_sw128(smem_u32(sDO), 16, 1024);            // dO stages, K-major
+    const uint64_t d_ones = sdesc_plain(smem_u32(sOnes), 128, 256);
+    const uint64_t d_qa = sdesc_plain(smem_u32(sQa), 128, 256);
+    const uint64_t d_da = sdesc_plain(smem_u32(sDa), 128, 256);
     bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
     tc_fence_after();
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b = st & 1, qs = st % QS, ds = st % DS;
+      const int qs = st % QS, ds = st % DS;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      // buffers b still feed dV(st-2) / dK(st-2), issued by the other warp
-      bool w = (st < 2 || mbar_wait(&acc_b[b], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
+      // the staging set is free once the row threads have loaded step st-1
+      bool w = (st < 1 || mbar_wait(st_free, (st - 1) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile), bd = sdesc_add(ddk, ds * C::kStageTile);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 64 * b, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+        umma_ss_w(tmem, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bq, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      umma_ss_w(tmem, d_ones, sdesc_add(d_qa, qs * kAugStage), idesc_s, 1u);
       if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (st / DS) & 1, ab))) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 128 + 64 * b, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+        umma_ss_w(tmem + 64, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_commit_w(&st_full[b]);
+      umma_ss_w(tmem + 64, d_ones, sdesc_add(d_da, ds * kAugStage), idesc_s, 1u);
+      umma_commit_w(st_full);
     }
     umma_commit_w(&drain[0]);
     mbar_wait_drain(&drain[0], 0);
@@ -272,12 +347,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile), bd = sdesc_add(ddm, ds * C::kStageTile);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
-        if (j < n) umma_ts_w(tDV, tmem + 64 * b + ds_col(j), sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+        if (j < n) umma_ts_w(tDV, tmem + 128 + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
       umma_commit_w(&do_empty[ds]);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
         if (j < n)
-          umma_ts_w(tDK, tmem + 128 + 64 * b + ds_col(j), sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+          umma_ts_w(tDK, tmem + 160 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
       umma_commit_w(&q_empty[qs]);
       umma_commit_w(&acc_b[b]);
     }
@@ -297,49 +372,37 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t mw[2];
     if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
-      const int b = st & 1, ds = st % DS;
+      const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
-      ok = mbar_wait(&st_full[b], (st >> 1) & 1, ab) && mbar_wait(&ld_full[ds], (st / DS) & 1, ab);
-      ok = __all_sync(0xffffffffu, ok);
+      ok = __all_sync(0xffffffffu, mbar_wait(st_full, st & 1, ab));
       if (!ok) break;
       tc_fence_after();
       uint32_t a[32], d[32];
       if (active) {
-        tmem_ld32(tmem + 64 * b + lane_off + grp * 32, a);
-        tmem_ld32(tmem + 128 + 64 * b + lane_off + grp * 32, d);
+        tmem_ld32(tmem + lane_off + grp * 32, a);
+        tmem_ld32(tmem + 64 + lane_off + grp * 32, d);
+        tmem_wait_ld();
       }
+      tc_fence_before();
+      mbar_arrive(st_free);
       uint32_t mw_next[2] = {0u, 0u};
       if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
+      // a = S^T - LSE/scale, d = dP^T - Delta (fp32, from the augmented MMAs)
+      uint32_t pp[16], pd[16];
       if (active) {
-        tmem_wait_ld();
         const uint32_t m = grp ? mw[1] : mw[0];
-        const float4* sl4 = reinterpret_cast<const float4*>(sLD + ds * 128 + grp * 32);
-        const float4* sd4 = reinterpret_cast<const float4*>(sLD + ds * 128 + 64 + grp * 32);
-        uint32_t pp[16], pd[16];
         if (m == 0xFFFFFFFFu) {
           // every column allowed: no masking, all values finite
 #pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 L = sl4[i4];
-            const float4 Dl = sd4[i4];
-            float p0, p1, p2, p3, s0, s1, s2, s3;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
-                             f2_pack(-L.x, -L.y)), p0, p1);
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
-                             f2_pack(-L.z, -L.w)), p2, p3);
-            p0 = ex2(p0);
-            p1 = ex2(p1);
-            p2 = ex2(p2);
-            p3 = ex2(p3);
-            f2_unpack(f2_mul(f2_pack(p0, p1), f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])),
-                                                      f2_pack(-Dl.x, -Dl.y))), s0, s1);
-            f2_unpack(f2_mul(f2_pack(p2, p3), f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
-                                                      f2_pack(-Dl.z, -Dl.w))), s2, s3);
-            pp[2 * i4] = pack_bf16(p0, p1);
-            pp[2 * i4 + 1] = pack_bf16(p2, p3);
-            pd[2 * i4] = pack_bf16(s0, s1);
-            pd[2 * i4 + 1] = pack_bf16(s2, s3);
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1, s0, s1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
+                      s1);
+            pp[i] = pack_bf16(p0, p1);
+            pd[i] = pack_bf16(s0, s1);
           }
         } else if (m == 0u) {
 #pragma unroll
@@ -349,35 +412,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
         } else {
 #pragma unroll
-          for (int i4 = 0; i4 < 8; ++i4) {
-            const float4 L = sl4[i4];
-            const float4 Dl = sd4[i4];
-            float x0, x1, x2, x3;
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4]), __uint_as_float(a[4 * i4 + 1])), sl2x2,
-                             f2_pack(-L.x, -L.y)), x0, x1);
-            f2_unpack(f2_fma(f2_pack(__uint_as_float(a[4 * i4 + 2]), __uint_as_float(a[4 * i4 + 3])), sl2x2,
-                             f2_pack(-L.z, -L.w)), x2, x3);
-            float p[4] = {ex2(x0), ex2(x1), ex2(x2), ex2(x3)};
-#pragma unroll
-            for (int h = 0; h < 4; ++h)
-              if (!((m >> (4 * i4 + h)) & 1u)) p[h] = 0.f;
-            float g0, g1, g2, g3;
-            f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4]), __uint_as_float(d[4 * i4 + 1])), f2_pack(-Dl.x, -Dl.y)),
-                      g0, g1);
-            f2_unpack(f2_add(f2_pack(__uint_as_float(d[4 * i4 + 2]), __uint_as_float(d[4 * i4 + 3])),
-                             f2_pack(-Dl.z, -Dl.w)), g2, g3);
-            float s0, s1, s2, s3;
-            f2_unpack(f2_mul(f2_pack(p[0], p[1]), f2_pack(g0, g1)), s0, s1);
-            f2_unpack(f2_mul(f2_pack(p[2], p[3]), f2_pack(g2, g3)), s2, s3);
-            pp[2 * i4] = pack_bf16(p[0], p[1]);
-            pp[2 * i4 + 1] = pack_bf16(p[2], p[3]);
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1, s0, s1;
+            f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
+            float p0 = ex2(x0), p1 = ex2(x1);
+            if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
+            if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
+            f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
+                      s1);
+            pp[i] = pack_bf16(p0, p1);
             // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
-            pd[2 * i4] = pack_bf16(p[0] != 0.f ? s0 : 0.f, p[1] != 0.f ? s1 : 0.f);
-            pd[2 * i4 + 1] = pack_bf16(p[2] != 0.f ? s2 : 0.f, p[3] != 0.f ? s3 : 0.f);
+            pd[i] = pack_bf16(p0 != 0.f ? s0 : 0.f, p1 != 0.f ? s1 : 0.f);
           }
         }
-        tmem_st16(tmem + 64 * b + lane_off + grp * 32, pp);
-        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 32, pd);
+      }
+      // Packed set b still feeds dV(st-2) / dK(st-2).  Every row thread waits,
+      // active or not, so that no arrival for step st can land in the
+      // pt_full phase of step st-2.
+      if (st >= 2 && !__all_sync(0xffffffffu, mbar_wait(&acc_b[b], ((st - 2) >> 1) & 1, ab))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (active) {
+        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 16, pp);
+        tmem_st16(tmem + 160 + 64 * b + lane_off + grp * 16, pd);
         tmem_wait_st();
       }
       tc_fence_before();
@@ -422,10 +481,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // K4: dQ (query-owned tiles, key pages as columns; the forward lists)
 // ----------------------------------------------------------------------------
 // TMEM columns: the owned Q rows as bf16 pairs at 0 (the A operand of
-// S = Q K^T, so that MMA reads only K from shared memory), S / dS triple
-// buffer at 64, 128, 192, dP double buffer at 256, 320, dQ at 384.  With three
-// S buffers the MMA that reuses one waits for the dQ of three steps back,
-// which has long finished.
+// S = Q K^T, so that MMA reads only K from shared memory), two fp32 staging
+// sets (S at 64 + 64b, dP at 192 + 64b), two packed bf16 dS sets at 320 + 32p,
+// dQ at 384.  A staging set is free as soon as the row threads have loaded
+// it; a packed set is reused after the dQ MMAs of two steps back.
 template <int D>
 struct DqCfg {
   static constexpr int kNch = D / 64;
@@ -457,10 +516,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* k_empty = k_full + KS;
   uint64_t* v_full = k_empty + KS;
   uint64_t* v_empty = v_full + VS;
-  uint64_t* sd_full = v_empty + VS;  // [2] S and dP of a step are ready
-  uint64_t* ds_full = sd_full + 2;   // [2] dS of a step is in TMEM
-  uint64_t* dq_done = ds_full + 2;   // [3] dQ MMAs of the steps using S buffer b finished
-  uint64_t* acc_done = dq_done + 3;
+  uint64_t* sd_full = v_empty + VS;  // [2] S and dP of a step are in staging set b
+  uint64_t* s_free = sd_full + 2;    // [2] the row threads have loaded staging set b
+  uint64_t* ds_full = s_free + 2;    // [2] dS of a step is in packed set p
+  uint64_t* dq_done = ds_full + 2;   // [2] dQ MMAs of the steps using packed set p finished
+  uint64_t* acc_done = dq_done + 2;
   uint64_t* drain = acc_done + 1;    // [2] one per issuing warp
   uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 2);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
@@ -485,9 +545,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sd_full[b], 1);
+      mbar_init(&s_free[b], 256);
       mbar_init(&ds_full[b], 256);
+      mbar_init(&dq_done[b], 1);
     }
-    for (int b = 0; b < 3; ++b) mbar_init(&dq_done[b], 1);
     mbar_init(acc_done, 1);
     mbar_init(&drain[0], 1);
     mbar_init(&drain[1], 1);
@@ -499,8 +560,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tslot;
   const uint32_t tQ = tmem, tDQ = tmem + 384;
-  auto tS = [&](int b3) { return tmem + 64 + 64 * b3; };
-  auto tDP = [&](int b2) { return tmem + 256 + 64 * b2; };
+  auto tS = [&](int b) { return tmem + 64 + 64 * b; };
+  auto tDP = [&](int b) { return tmem + 192 + 64 * b; };
+  auto tPk = [&](int p) { return tmem + 320 + 32 * p; };
 
   if (warp == 0) {
     // ---------------- producer (whole warp; lane j owns page j of a step) ----------------
@@ -545,28 +607,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab) && mbar_wait(q_ready, 0, ab));
     tc_fence_after();
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b2 = st & 1, b3 = st % 3, ks = st % KS, vs = st % VS;
+      const int b = st & 1, ks = st % KS, vs = st % VS;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      // S buffer b3 still feeds dQ(st-3) (issued by the other warp); per-buffer
-      // barrier, waited in order
-      bool w = (st < 3 || mbar_wait(&dq_done[b3], ((st / 3) - 1) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
+      // staging set b is free once the row threads have loaded step st-2
+      bool w = (st < 2 || mbar_wait(&s_free[b], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
       const uint64_t bk = sdesc_add(dkk, ks * C::kStageTile), bv = sdesc_add(dvk, vs * C::kStageTile);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ts_w(tS(b3), tQ + 8 * kk, sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      // dP buffer b2 is free once the row threads finished step st-2
-      w = (st < 2 || mbar_wait(&ds_full[b2], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&v_full[vs], (st / VS) & 1, ab);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        umma_ts_w(tS(b), tQ + 8 * kk, sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+      if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (st / VS) & 1, ab))) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tDP(b2), sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+        umma_ss_w(tDP(b), sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bv, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
       umma_commit_w(&v_empty[vs]);
-      umma_commit_w(&sd_full[b2]);
+      umma_commit_w(&sd_full[b]);
     }
     umma_commit_w(&drain[0]);
     mbar_wait_drain(&drain[0], 0);
@@ -576,16 +635,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
     bool ok = true;
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b2 = st & 1, b3 = st % 3, ks = st % KS;
-      if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[b2], (st >> 1) & 1, ab))) { ok = false; break; }
+      const int p = st & 1, ks = st % KS;
+      if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[p], (st >> 1) & 1, ab))) { ok = false; break; }
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
       const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
-        if (j < n) umma_ts_w(tDQ, tS(b3) + ds_col(j), sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+        if (j < n) umma_ts_w(tDQ, tPk(p) + 8 * j, sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
       umma_commit_w(&k_empty[ks]);
-      umma_commit_w(&dq_done[b3]);
+      umma_commit_w(&dq_done[p]);
     }
     if (ok && n_steps > 0) umma_commit_w(acc_done);
     umma_commit_w(&drain[1]);
@@ -638,23 +697,25 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint32_t mw[2];
     if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
     for (int st = 0; st < n_steps; ++st) {
-      const int b2 = st & 1, b3 = st % 3;
+      const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b2], (st >> 1) & 1, ab));
+      ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
       uint32_t a[32], d[32];
       if (active) {
-        tmem_ld32(tS(b3) + lane_off + grp * 32, a);
-        tmem_ld32(tDP(b2) + lane_off + grp * 32, d);
+        tmem_ld32(tS(b) + lane_off + grp * 32, a);
+        tmem_ld32(tDP(b) + lane_off + grp * 32, d);
+        tmem_wait_ld();
       }
+      tc_fence_before();
+      mbar_arrive(&s_free[b]);
       uint32_t mw_next[2] = {0u, 0u};
       if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
+      uint32_t pd[16];
       if (active) {
-        tmem_wait_ld();
         const uint32_t m = grp ? mw[1] : mw[0];
-        uint32_t pd[16];
         if (m == 0xFFFFFFFFu) {
           // every column allowed: no masking, all values finite
 #pragma unroll
@@ -683,11 +744,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             pd[i] = pack_bf16(p0 != 0.f ? g0 : 0.f, p1 != 0.f ? g1 : 0.f);
           }
         }
-        tmem_st16(tS(b3) + lane_off + grp * 32, pd);
+      }
+      // Packed set b still feeds dQ(st-2).  Every row thread waits, active or
+      // not: dq_done(st-2) implies that ds_full finished the phase of step
+      // st-2, so no thread can arrive for step st while that phase is open.
+      if (st >= 2 && !__all_sync(0xffffffffu, mbar_wait(&dq_done[b], ((st - 2) >> 1) & 1, ab))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (active) {
+        tmem_st16(tPk(b) + lane_off + grp * 16, pd);
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&ds_full[b2]);
+      mbar_arrive(&ds_full[b]);
       mw[0] = mw_next[0];
       mw[1] = mw_next[1];
     }
@@ -740,7 +811,7 @@ static cudaError_t launch_dkdv_t(const TmaPages& tk, const TmaPages& tv, const T
   using C = DkvCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
-  dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), kBwdThreads, C::kSmem, st>>>(
+  dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), kDkvThreads, C::kSmem, st>>>(
       tk, tv, tq, tdo, a.work, a.pages, a.masks, lse, delta, dk, dv, a.own_slots, a.col_slots, a.scale * kLog2e,
       a.scale, a.err);
   return cudaGetLastError();

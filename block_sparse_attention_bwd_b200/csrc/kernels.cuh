@@ -15,6 +15,10 @@ namespace spattn {
 // page-sized box in about the same time.
 struct TmaPages {
   CUtensorMap m16, m32, m64;
+  // 64 rows x every 64-column chunk in one request (4D map: columns, rows,
+  // chunk, batch*head); it lands chunk after chunk, 8 KB apart, which is the
+  // layout of a 64-row stage.  Equal to m64 when head_dim is 64.
+  CUtensorMap m64w;
 };
 
 // Everything one attention launch needs besides its tensor maps.

@@ -59,7 +59,10 @@ __device__ __forceinline__ void step_masks(const uint64_t* __restrict__ masks, i
 // chunks are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every
 // chunk.  Lane j < n holds page id `pid` of page j.  Maximal runs of
 // consecutive page ids are fetched with 64-, 32- and 16-row boxes by the
-// run's first lane.  All 32 lanes must call this.
+// run's first lane; a run that fills a whole 64-row stage (chunks 8 KB
+// apart) takes one request for all chunks.  Each TMA request costs the
+// issuing thread time whatever its size, so fewer, larger boxes keep the
+// producer off the critical path.  All 32 lanes must call this.
 template <int NCH>
 __device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, const TmaPages& maps, int pid, int n,
                                                int bh, uint64_t* bar) {
@@ -70,6 +73,11 @@ __device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, co
   if (!start) return;
   int rem = __ffs(~(cont >> lane));  // run length
   int j = lane;
+  if (NCH > 1 && lane == 0 && rem >= 4 && chunk_bytes == 64 * 128) {
+    tma_load_4d(dst, &maps.m64w, 0, pid * 16, 0, bh, bar);
+    j += 4;
+    rem -= 4;
+  }
   auto box = [&](const CUtensorMap* m, int rows) {
 #pragma unroll
     for (int c = 0; c < NCH; ++c)
