@@ -108,19 +108,19 @@ struct DkvCfg {
   static constexpr int kSmem = 2 * kTile + (kQStages + kDStages) * (kStageTile + kAugStage) + kOnesBytes + 1024 + 512;
 };
 
-// 11 warps: 0 = TMA producer, 1 = TMEM owner and issuer of the MMAs that
-// read the step's column tiles into TMEM (S^T/dP^T or S/dP), 2..9 = two
+// 12 warps: 0 and 11 = TMA producers, 1 = TMEM owner and issuer of the MMAs
+// that read the step's column tiles into TMEM (S^T/dP^T or S/dP), 2..9 = two
 // groups of row threads, 10 = issuer of the accumulating MMAs (dV/dK or dQ).
 // Row group g (warps 2+4g .. 5+4g) handles columns 32g .. 32g+31 of every
 // 64-column step (warp w reaches TMEM lanes of quarter w%4).  The tensor
 // core accepts only a couple of MMAs ahead of the one it runs, so a single
 // issuing warp idles it whenever that warp waits; with two issuers one keeps
 // it busy while the other waits.
-constexpr int kBwdThreads = 352;
 constexpr int kAccWarp = 10;
-// dK / dV add warp 11, the producer of the dO stages (warp 0 produces the Q
-// stages): a TMA request holds its issuing thread for hundreds of cycles, so
-// one producer for both column tensors would set the step time.
+// Warp 11 is the second producer (dO stages for dK / dV, V stages for dQ;
+// warp 0 produces the Q or K stages): a TMA request holds its issuing thread
+// for hundreds of cycles, so one producer for both column tensors would set
+// the step time.
 constexpr int kDkvThreads = 384;
 constexpr int kDoWarp = 11;
 
@@ -369,12 +369,16 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const int seg = code < 4 ? static_cast<int>(code) : -1;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
-    uint32_t mw[2];
-    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
+    StepMasks<NP> raw;
+    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols));
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
+      uint32_t mw[2];
+      raw.bits(seg, mw);
+      // mask words of the next step load while this one computes
+      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP));
       ok = __all_sync(0xffffffffu, mbar_wait(st_full, st & 1, ab));
       if (!ok) break;
       tc_fence_after();
@@ -386,8 +390,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(st_free);
-      uint32_t mw_next[2] = {0u, 0u};
-      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
       // a = S^T - LSE/scale, d = dP^T - Delta (fp32, from the augmented MMAs)
       uint32_t pp[16], pd[16];
       if (active) {
@@ -441,8 +443,6 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&pt_full[b]);
-      mw[0] = mw_next[0];
-      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, ab));
@@ -496,7 +496,7 @@ struct DqCfg {
 };
 
 template <int D>
-__global__ void __launch_bounds__(kBwdThreads, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     dq_kernel(const __nv_bfloat16* __restrict__ q, const __grid_constant__ TmaPages tm_do,
               const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
               const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
@@ -564,40 +564,46 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   auto tDP = [&](int b) { return tmem + 192 + 64 * b; };
   auto tPk = [&](int p) { return tmem + 320 + 32 * p; };
 
-  if (warp == 0) {
-    // ---------------- producer (whole warp; lane j owns page j of a step) ----------------
+  if (warp == 0 || warp == kDoWarp) {
+    // ---------------- producers (whole warps): warp 0 = K stages, warp 11 = V stages ----------------
+    // Lane j owns page j of a step; page ids are fetched one step ahead.
+    const bool is_k = warp == 0;
+    const int NS = is_k ? KS : VS;
+    uint8_t* stage0 = is_k ? sK : sV;
+    uint64_t* full = is_k ? k_full : v_full;
+    uint64_t* empty = is_k ? k_empty : v_empty;
+    const TmaPages& tm = is_k ? tm_k : tm_v;
+    if (is_k) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_do.m64);
+        mbar_arrive_expect_tx(own_full, wk.n_own * C::kNch * 2048);
+      }
+      __syncwarp();
+      load_page_runs<C::kNch>(sDO, kChunkBytes, tm_do, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh,
+                              own_full);
+    }
     if (lane == 0) {
-      tma_prefetch_desc(&tm_do.m64);
-      tma_prefetch_desc(&tm_k.m64);
-      tma_prefetch_desc(&tm_v.m64);
-      mbar_arrive_expect_tx(own_full, wk.n_own * C::kNch * 2048);
+      tma_prefetch_desc(&tm.m64w);
+      tma_prefetch_desc(&tm.m64);
     }
     __syncwarp();
-    load_page_runs<C::kNch>(sDO, kChunkBytes, tm_do, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh,
-                            own_full);
     int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
-    int k_issued = 0, v_issued = 0;
+    int issued = 0;
     for (int st = 0; st < n_steps; ++st) {
-      const int ks = st % KS, vs = st % VS;
+      const int s = st % NS;
       const int n = min(NP, n_cols - st * NP);
       const int pid = pid_next;
       if (st + 1 < n_steps)
         pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
-      if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+      if (st >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / NS) - 1) & 1, ab))) break;
+      if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(sK + ks * C::kStageTile, kStageChunk, tm_k, pid, n, wk.bh, &k_full[ks]);
-      k_issued = st + 1;
-      if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
-      __syncwarp();
-      load_page_runs<C::kNch>(sV + vs * C::kStageTile, kStageChunk, tm_v, pid, n, wk.bh, &v_full[vs]);
-      v_issued = st + 1;
+      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
+      issued = st + 1;
     }
     if (lane == 0) {
-      for (int st = max(0, k_issued - KS); st < k_issued; ++st) mbar_wait_drain(&k_full[st % KS], (st / KS) & 1);
-      for (int st = max(0, v_issued - VS); st < v_issued; ++st) mbar_wait_drain(&v_full[st % VS], (st / VS) & 1);
-      mbar_wait_drain(own_full, 0);
+      for (int st = max(0, issued - NS); st < issued; ++st) mbar_wait_drain(&full[st % NS], (st / NS) & 1);
+      if (is_k) mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
     // ---------------- S, dP issuer (warp-wide; one elected lane issues) ----------------
@@ -694,12 +700,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t nl2 = f2_pack(-lse2, -lse2);
     const uint64_t ndl = f2_pack(-dl, -dl);
     bool ok = true;
-    uint32_t mw[2];
-    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
+    StepMasks<NP> raw;
+    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols));
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
+      uint32_t mw[2];
+      raw.bits(seg, mw);
+      // mask words of the next step load while this one computes
+      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP));
       ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
@@ -711,8 +721,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&s_free[b]);
-      uint32_t mw_next[2] = {0u, 0u};
-      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
       uint32_t pd[16];
       if (active) {
         const uint32_t m = grp ? mw[1] : mw[0];
@@ -759,8 +767,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&ds_full[b]);
-      mw[0] = mw_next[0];
-      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, ab));
@@ -824,7 +830,7 @@ static cudaError_t launch_dq_t(const __nv_bfloat16* q, const TmaPages& tdo, cons
   using C = DqCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
-  dq_kernel<D><<<static_cast<unsigned>(a.n_work), kBwdThreads, C::kSmem, st>>>(
+  dq_kernel<D><<<static_cast<unsigned>(a.n_work), kDkvThreads, C::kSmem, st>>>(
       q, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.err);
   return cudaGetLastError();
 }

@@ -206,11 +206,15 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
-    uint32_t mw[2];
-    if (n_steps > 0) step_masks<NP>(col_masks, wk.e0, min(NP, n_cols), seg, mw);
+    StepMasks<NP> raw;
+    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols));
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
+      uint32_t mw[2];
+      raw.bits(seg, mw);
+      // mask words of the next step load while this one computes
+      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP));
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
@@ -218,9 +222,6 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
 #pragma unroll
       for (int pc = 0; pc < 2; ++pc)
         if (pc * 32 < N) tmem_ld32(tmem + 64 * b + lane_off + pc * 32, sr[pc]);
-      // masks of the next step load while this one computes
-      uint32_t mw_next[2] = {0u, 0u};
-      if (st + 1 < n_steps) step_masks<NP>(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg, mw_next);
       tmem_wait_ld();
       // masked row max over four independent chains
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
@@ -299,8 +300,6 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(&p_full[b]);
-      mw[0] = mw_next[0];
-      mw[1] = mw_next[1];
     }
     if (ok && n_steps > 0) {
       ok = mbar_wait(o_done, (n_steps - 1) & 1, ab);

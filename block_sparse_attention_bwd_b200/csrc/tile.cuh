@@ -38,22 +38,31 @@ __device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {
   return x;
 }
 
-// Row mask of one step of NP pages: bit c of word c/32 <=> column c of the
-// step may be attended by this row.  `seg` < 0 gives an all-zero mask.
+// The column-list mask words of one step of NP pages (16 bits per segment
+// per page).  `fetch` only issues the loads; the words are read by `bits`,
+// an iteration later, so the load latency never stalls the row math that
+// runs in between.
 template <int NP>
-__device__ __forceinline__ void step_masks(const uint64_t* __restrict__ masks, int first, int n, int seg,
-                                           uint32_t (&mw)[NP / 2]) {
+struct StepMasks {
+  uint64_t w[NP];
+  __device__ __forceinline__ void fetch(const uint64_t* __restrict__ masks, int first, int n) {
 #pragma unroll
-  for (int i = 0; i < NP / 2; ++i) mw[i] = 0u;
-  if (seg < 0) return;
-#pragma unroll
-  for (int j = 0; j < NP; ++j) {
-    if (j < n) {
-      const uint32_t bits = static_cast<uint32_t>(__ldg(masks + first + j) >> (16 * seg)) & 0xFFFFu;
-      mw[j >> 1] |= bits << (16 * (j & 1));
+    for (int j = 0; j < NP; ++j) {
+      w[j] = 0ull;
+      if (j < n) w[j] = __ldg(masks + first + j);
     }
   }
-}
+  // Row mask of the step: bit c of word c/32 <=> column c may be attended by
+  // a row of segment `seg`; `seg` < 0 gives an all-zero mask.
+  __device__ __forceinline__ void bits(int seg, uint32_t (&mw)[NP / 2]) const {
+#pragma unroll
+    for (int i = 0; i < NP / 2; ++i) mw[i] = 0u;
+    if (seg < 0) return;
+#pragma unroll
+    for (int j = 0; j < NP; ++j)
+      mw[j >> 1] |= (static_cast<uint32_t>(w[j] >> (16 * seg)) & 0xFFFFu) << (16 * (j & 1));
+  }
+};
 
 // Warp-collective TMA gather of n (<= 32) pages into a stage whose 64-column
 // chunks are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every
