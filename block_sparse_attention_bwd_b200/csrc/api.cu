@@ -53,13 +53,13 @@ bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64
 // every chunk of those rows, chunk after chunk.  The chunk stride (128 B) is
 // below the row stride; a tiled map only needs each stride to be a multiple
 // of 16 bytes.
-bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows) {
   auto fn = encode_fn();
   if (!fn) return false;
   const int nch = head_dim / 64;
   cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nch), static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[3] = {static_cast<cuuint64_t>(head_dim) * 2, 128, static_cast<cuuint64_t>(head_dim) * 2 * rows};
-  cuuint32_t box[4] = {64, 64, static_cast<cuuint32_t>(nch), 1};
+  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(nch), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -70,11 +70,12 @@ bool make_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_
   if (!make_map(&t->m16, ptr, head_dim, rows, bh, 16) || !make_map(&t->m32, ptr, head_dim, rows, bh, 32) ||
       !make_map(&t->m64, ptr, head_dim, rows, bh, 64))
     return false;
+  if (!make_wide_map(&t->m128w, ptr, head_dim, rows, bh, 128)) return false;
   if (head_dim == 64) {
     t->m64w = t->m64;
     return true;
   }
-  return make_wide_map(&t->m64w, ptr, head_dim, rows, bh);
+  return make_wide_map(&t->m64w, ptr, head_dim, rows, bh, 64);
 }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

@@ -71,6 +71,12 @@ __global__ void delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfl
 // compute step c; the packed set of step c is reused two steps later, after
 // the dV / dK MMAs that read it.
 //
+// Column tiles arrive in stages of one 64-column MMA step (dK / dV) or two
+// (dQ, 128 rows, one 32 KB box): a TMA request holds its issuing thread for
+// a long time whatever its size, so larger stages keep a producer ahead of the
+// tensor core, while more stages give more slack between a stage's release
+// and its reuse; dK / dV have room for four 64-row stages per tensor only.
+//
 // The per-column terms of the backward pass are folded into the two MMAs
 // with one extra K = 16 slice each, so the row threads read nothing but
 // TMEM: with x = LSE / scale of query column c, split into three bf16 terms
@@ -79,10 +85,9 @@ __global__ void delta_kernel(const __nv_bfloat16* __restrict__ o, const __nv_bfl
 //   [V | 1 1 1 0..] . [dO | -Delta split]^T = dP^T - Delta,
 // both accumulated in fp32.  The slices are 16 bf16 wide, in the plain
 // (unswizzled) K-major layout: a 128-row block of ones shared by both MMAs,
-// and one 64-row block per Q / dO stage that the producer writes.
-constexpr int kBwdStepPages = 4;                  // 64 columns per step
-constexpr int kStageChunk = 64 * 128;             // one 64-column chunk of a 64-row stage
-constexpr int kAugStage = 64 * 32;                // 64 rows x 16 bf16, plain layout
+// and one block per Q / dO stage that the producer writes.
+constexpr int kBwdStepPages = 4;                  // 64 columns per MMA step
+constexpr int kHalfStage = 64 * 128;              // offset of a two-step stage's second step in a chunk
 constexpr int kOnesBytes = 128 * 32;              // 128 rows x 16 bf16, plain layout
 
 // Byte offset of row r (first 8 of its 16 elements) in a plain K-major
@@ -102,7 +107,10 @@ template <int D>
 struct DkvCfg {
   static constexpr int kNch = D / 64;
   static constexpr int kTile = kNch * kChunkBytes;     // owned 128-row tile
-  static constexpr int kStageTile = kNch * kStageChunk;  // 64-row column stage
+  static constexpr int kStagePages = 4;                  // one step per stage
+  static constexpr int kStageChunk = kStagePages * 16 * 128;  // one 64-column chunk of a stage
+  static constexpr int kStageTile = kNch * kStageChunk;
+  static constexpr int kAugStage = kStagePages * 16 * 32;     // plain-layout slice of a stage
   static constexpr int kQStages = (D == 128) ? 4 : 6;
   static constexpr int kDStages = (D == 128) ? 4 : 6;
   static constexpr int kSmem = 2 * kTile + (kQStages + kDStages) * (kStageTile + kAugStage) + kOnesBytes + 1024 + 512;
@@ -134,7 +142,10 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                 __nv_bfloat16* __restrict__ out_dv, int64_t kv_slots, int64_t q_slots, float sl2, float scale,
                 int* err) {
   using C = DkvCfg<D>;
-  constexpr int QS = C::kQStages, DS = C::kDStages, NP = kBwdStepPages;
+  constexpr int QS = C::kQStages, DS = C::kDStages, NP = kBwdStepPages, SP = C::kStagePages;
+  constexpr int SPS = SP / NP;       // steps per stage
+  constexpr int NH = SP * 16 / 32;  // stage columns per producer lane
+  constexpr int kStageChunk = C::kStageChunk, kAugStage = C::kAugStage;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sK = smem;
@@ -233,27 +244,28 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       tma_prefetch_desc(&tm.m64w);
       tma_prefetch_desc(&tm.m64);
     }
-    // Lane j holds the page id of column page j of steps st and st+1, and the
-    // per-column term (LSE for Q, Delta for dO) of columns lane and lane+32 of
-    // step st.  Both are fetched one step ahead, and the fetched values are
+    // Lane j holds the page id of column page j of stages t and t+1, and the
+    // per-column term (LSE for Q, Delta for dO) of columns lane + 32h of
+    // stage t.  Both are fetched one stage ahead, and the fetched values are
     // used only in the next iteration, so their global-load latency overlaps
     // the waits and TMA issue of the current one instead of stalling it.
     const float inv_scale = 1.0f / scale;
-    auto page_id = [&](int s) {
-      return (s < n_steps && lane < min(NP, n_cols - s * NP)) ? __ldg(col_pages + wk.e0 + s * NP + lane) : 0;
+    const int n_stages = (n_cols + SP - 1) / SP;
+    auto page_id = [&](int t) {
+      return (t < n_stages && lane < min(SP, n_cols - t * SP)) ? __ldg(col_pages + wk.e0 + t * SP + lane) : 0;
     };
     // Raw loads only (nothing here reads the loaded registers); a dead column
     // (beyond the step or the tensor) loads a valid address and is zeroed
     // where the value is used, through its bit in `live`.
-    auto fetch_terms = [&](int s, int pg_lane, float (&x)[2], uint32_t& live) {
-      const int n_s = min(NP, n_cols - s * NP);
+    auto fetch_terms = [&](int t, int pg_lane, float (&x)[NH], uint32_t& live) {
+      const int n_t = min(SP, n_cols - t * SP);
       live = 0u;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int idx = lane + 32 * h;  // column of the step
+      for (int h = 0; h < NH; ++h) {
+        const int idx = lane + 32 * h;  // column of the stage
         const int pg = __shfl_sync(0xffffffffu, pg_lane, idx >> 4);
         const int64_t slot = static_cast<int64_t>(pg) * 16 + (idx & 15);
-        const bool ok = s < n_steps && (idx >> 4) < n_s && slot < q_slots;
+        const bool ok = t < n_stages && (idx >> 4) < n_t && slot < q_slots;
         x[h] = __ldg(terms + static_cast<int64_t>(wk.bh) * q_slots + (ok ? slot : 0));
         live |= ok ? (1u << h) : 0u;
       }
@@ -266,35 +278,35 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       return aug_row(ok && isfinite(x) ? x : 0.f);
     };
     int pid = page_id(0), pid_next = page_id(1);
-    float xc[2];
+    float xc[NH];
     uint32_t livec;
     fetch_terms(0, pid, xc, livec);
     int issued = 0;
-    for (int st = 0; st < n_steps; ++st) {
-      const int s = st % NS;
-      const int n = min(NP, n_cols - st * NP);
-      const int pid_next2 = page_id(st + 2);
-      float xn[2];
+    for (int t = 0; t < n_stages; ++t) {
+      const int s = t % NS;
+      const int n = min(SP, n_cols - t * SP);
+      const int pid_next2 = page_id(t + 2);
+      float xn[NH];
       uint32_t liven;
-      fetch_terms(st + 1, pid_next, xn, liven);
-      if (st >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / NS) - 1) & 1, ab))) break;
+      fetch_terms(t + 1, pid_next, xn, liven);
+      if (t >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((t / NS) - 1) & 1, ab))) break;
 #pragma unroll
-      for (int h = 0; h < 2; ++h)
+      for (int h = 0; h < NH; ++h)
         *reinterpret_cast<uint4*>(aug0 + s * kAugStage + aug_row_off(lane + 32 * h)) = term_row(xc[h], (livec >> h) & 1u);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
       __syncwarp();
       load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
-      issued = st + 1;
+      issued = t + 1;
       pid = pid_next;
       pid_next = pid_next2;
       livec = liven;
-      xc[0] = xn[0];
-      xc[1] = xn[1];
+#pragma unroll
+      for (int h = 0; h < NH; ++h) xc[h] = xn[h];
     }
     if (lane == 0) {
-      for (int st = max(0, issued - NS); st < issued; ++st) mbar_wait_drain(&full[st % NS], (st / NS) & 1);
+      for (int t = max(0, issued - NS); t < issued; ++t) mbar_wait_drain(&full[t % NS], (t / NS) & 1);
       if (is_q) mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
@@ -309,26 +321,27 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
     tc_fence_after();
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int qs = st % QS, ds = st % DS;
+      const int t = st / SPS, half = st % SPS, qs = t % QS, ds = t % DS;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
       // the staging set is free once the row threads have loaded step st-1
-      bool w = (st < 1 || mbar_wait(st_free, (st - 1) & 1, ab)) && mbar_wait(&q_full[qs], (st / QS) & 1, ab);
+      bool w = (st < 1 || mbar_wait(st_free, (st - 1) & 1, ab)) && mbar_wait(&q_full[qs], (t / QS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile), bd = sdesc_add(ddk, ds * C::kStageTile);
+      const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile + half * kHalfStage);
+      const uint64_t bd = sdesc_add(ddk, ds * C::kStageTile + half * kHalfStage);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
         umma_ss_w(tmem, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bq, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_ss_w(tmem, d_ones, sdesc_add(d_qa, qs * kAugStage), idesc_s, 1u);
-      if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (st / DS) & 1, ab))) { ok = false; break; }
+      umma_ss_w(tmem, d_ones, sdesc_add(d_qa, qs * kAugStage + half * 2048), idesc_s, 1u);
+      if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (t / DS) & 1, ab))) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
         umma_ss_w(tmem + 64, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_ss_w(tmem + 64, d_ones, sdesc_add(d_da, ds * kAugStage), idesc_s, 1u);
+      umma_ss_w(tmem + 64, d_ones, sdesc_add(d_da, ds * kAugStage + half * 2048), idesc_s, 1u);
       umma_commit_w(st_full);
     }
     umma_commit_w(&drain[0]);
@@ -340,20 +353,23 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
     bool ok = true;
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b = st & 1, qs = st % QS, ds = st % DS;
+      const int b = st & 1, t = st / SPS, half = st % SPS, qs = t % QS, ds = t % DS;
+      // a stage is released after the MMAs of its last step
+      const bool stage_end = half == SPS - 1 || st + 1 == n_steps;
       if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (st >> 1) & 1, ab))) { ok = false; break; }
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
-      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile), bd = sdesc_add(ddm, ds * C::kStageTile);
+      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile + half * kHalfStage);
+      const uint64_t bd = sdesc_add(ddm, ds * C::kStageTile + half * kHalfStage);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
         if (j < n) umma_ts_w(tDV, tmem + 128 + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&do_empty[ds]);
+      if (stage_end) umma_commit_w(&do_empty[ds]);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
         if (j < n)
           umma_ts_w(tDK, tmem + 160 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&q_empty[qs]);
+      if (stage_end) umma_commit_w(&q_empty[qs]);
       umma_commit_w(&acc_b[b]);
     }
     if (ok && n_steps > 0) umma_commit_w(acc_done);
@@ -489,9 +505,11 @@ template <int D>
 struct DqCfg {
   static constexpr int kNch = D / 64;
   static constexpr int kTile = kNch * kChunkBytes;        // dO tile (128 rows)
-  static constexpr int kStageTile = kNch * kStageChunk;   // 64-row K / V stage
-  static constexpr int kKStages = (D == 128) ? 6 : 10;
-  static constexpr int kVStages = (D == 128) ? 5 : 10;
+  static constexpr int kStagePages = 8;                   // two steps per stage
+  static constexpr int kStageChunk = kStagePages * 16 * 128;
+  static constexpr int kStageTile = kNch * kStageChunk;   // 128-row K / V stage
+  static constexpr int kKStages = (D == 128) ? 3 : 5;
+  static constexpr int kVStages = (D == 128) ? 3 : 5;
   static constexpr int kSmem = kTile + (kKStages + kVStages) * kStageTile + 1024 + 512;
 };
 
@@ -503,7 +521,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
               const uint64_t* __restrict__ col_masks, const float* __restrict__ lse, const float* __restrict__ delta,
               __nv_bfloat16* __restrict__ out_dq, int64_t q_slots, float sl2, float scale, int* err) {
   using C = DqCfg<D>;
-  constexpr int KS = C::kKStages, VS = C::kVStages, NP = kBwdStepPages;
+  constexpr int KS = C::kKStages, VS = C::kVStages, NP = kBwdStepPages, SP = C::kStagePages;
+  constexpr int SPS = SP / NP;  // steps per stage
+  constexpr int kStageChunk = C::kStageChunk;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sDO = smem;
@@ -566,7 +586,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 
   if (warp == 0 || warp == kDoWarp) {
     // ---------------- producers (whole warps): warp 0 = K stages, warp 11 = V stages ----------------
-    // Lane j owns page j of a step; page ids are fetched one step ahead.
+    // Lane j owns page j of a 128-row stage; page ids are fetched one stage
+    // ahead.
     const bool is_k = warp == 0;
     const int NS = is_k ? KS : VS;
     uint8_t* stage0 = is_k ? sK : sV;
@@ -587,22 +608,23 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       tma_prefetch_desc(&tm.m64);
     }
     __syncwarp();
-    int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
+    const int n_stages = (n_cols + SP - 1) / SP;
+    int pid_next = (n_stages > 0 && lane < min(SP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int issued = 0;
-    for (int st = 0; st < n_steps; ++st) {
-      const int s = st % NS;
-      const int n = min(NP, n_cols - st * NP);
+    for (int t = 0; t < n_stages; ++t) {
+      const int s = t % NS;
+      const int n = min(SP, n_cols - t * SP);
       const int pid = pid_next;
-      if (st + 1 < n_steps)
-        pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
-      if (st >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((st / NS) - 1) & 1, ab))) break;
+      if (t + 1 < n_stages)
+        pid_next = lane < min(SP, n_cols - (t + 1) * SP) ? __ldg(col_pages + wk.e0 + (t + 1) * SP + lane) : 0;
+      if (t >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((t / NS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
       __syncwarp();
       load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
-      issued = st + 1;
+      issued = t + 1;
     }
     if (lane == 0) {
-      for (int st = max(0, issued - NS); st < issued; ++st) mbar_wait_drain(&full[st % NS], (st / NS) & 1);
+      for (int t = max(0, issued - NS); t < issued; ++t) mbar_wait_drain(&full[t % NS], (t / NS) & 1);
       if (is_k) mbar_wait_drain(own_full, 0);
     }
   } else if (warp == 1) {
@@ -613,24 +635,26 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab) && mbar_wait(q_ready, 0, ab));
     tc_fence_after();
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int b = st & 1, ks = st % KS, vs = st % VS;
+      const int b = st & 1, t = st / SPS, half = st % SPS, ks = t % KS, vs = t % VS;
+      const bool stage_end = half == SPS - 1 || st + 1 == n_steps;
       const int n = min(NP, n_cols - st * NP);
       const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
       // staging set b is free once the row threads have loaded step st-2
-      bool w = (st < 2 || mbar_wait(&s_free[b], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&k_full[ks], (st / KS) & 1, ab);
+      bool w = (st < 2 || mbar_wait(&s_free[b], ((st - 2) >> 1) & 1, ab)) && mbar_wait(&k_full[ks], (t / KS) & 1, ab);
       if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
       tc_fence_after();
-      const uint64_t bk = sdesc_add(dkk, ks * C::kStageTile), bv = sdesc_add(dvk, vs * C::kStageTile);
+      const uint64_t bk = sdesc_add(dkk, ks * C::kStageTile + half * kHalfStage);
+      const uint64_t bv = sdesc_add(dvk, vs * C::kStageTile + half * kHalfStage);
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
         umma_ts_w(tS(b), tQ + 8 * kk, sdesc_add(bk, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (st / VS) & 1, ab))) { ok = false; break; }
+      if (!__all_sync(0xffffffffu, mbar_wait(&v_full[vs], (t / VS) & 1, ab))) { ok = false; break; }
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk)
         umma_ss_w(tDP(b), sdesc_add(ddo0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
                   sdesc_add(bv, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_commit_w(&v_empty[vs]);
+      if (stage_end) umma_commit_w(&v_empty[vs]);
       umma_commit_w(&sd_full[b]);
     }
     umma_commit_w(&drain[0]);
@@ -641,15 +665,16 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
     bool ok = true;
     for (int st = 0; ok && st < n_steps; ++st) {
-      const int p = st & 1, ks = st % KS;
+      const int p = st & 1, t = st / SPS, half = st % SPS, ks = t % KS;
+      const bool stage_end = half == SPS - 1 || st + 1 == n_steps;
       if (!__all_sync(0xffffffffu, mbar_wait(&ds_full[p], (st >> 1) & 1, ab))) { ok = false; break; }
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
-      const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile);
+      const uint64_t bk = sdesc_add(dkm, ks * C::kStageTile + half * kHalfStage);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
         if (j < n) umma_ts_w(tDQ, tPk(p) + 8 * j, sdesc_add(bk, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      umma_commit_w(&k_empty[ks]);
+      if (stage_end) umma_commit_w(&k_empty[ks]);
       umma_commit_w(&dq_done[p]);
     }
     if (ok && n_steps > 0) umma_commit_w(acc_done);

@@ -19,6 +19,9 @@ struct TmaPages {
   // chunk, batch*head); it lands chunk after chunk, 8 KB apart, which is the
   // layout of a 64-row stage.  Equal to m64 when head_dim is 64.
   CUtensorMap m64w;
+  // The same 4D view with 128-row boxes: a whole 128-row stage or owned tile
+  // (chunks 16 KB apart) in one request.
+  CUtensorMap m128w;
 };
 
 // Everything one attention launch needs besides its tensor maps.

@@ -69,7 +69,8 @@ struct StepMasks {
 // chunk.  Lane j < n holds page id `pid` of page j.  Maximal runs of
 // consecutive page ids are fetched with 64-, 32- and 16-row boxes by the
 // run's first lane; a run that fills a whole 64-row stage (chunks 8 KB
-// apart) takes one request for all chunks.  Each TMA request costs the
+// apart) or a whole 128-row stage or tile (chunks 16 KB apart) takes one
+// request for all chunks.  Each TMA request costs the
 // issuing thread time whatever its size, so fewer, larger boxes keep the
 // producer off the critical path.  All 32 lanes must call this.
 template <int NCH>
@@ -82,7 +83,11 @@ __device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, co
   if (!start) return;
   int rem = __ffs(~(cont >> lane));  // run length
   int j = lane;
-  if (NCH > 1 && lane == 0 && rem >= 4 && chunk_bytes == 64 * 128) {
+  if (lane == 0 && rem >= 8 && chunk_bytes == 128 * 128) {
+    tma_load_4d(dst, &maps.m128w, 0, pid * 16, 0, bh, bar);
+    j += 8;
+    rem -= 8;
+  } else if (NCH > 1 && lane == 0 && rem >= 4 && chunk_bytes == 64 * 128) {
     tma_load_4d(dst, &maps.m64w, 0, pid * 16, 0, bh, bar);
     j += 4;
     rem -= 4;
