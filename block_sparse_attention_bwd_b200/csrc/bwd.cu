@@ -386,15 +386,15 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
     StepMasks<NP> raw;
-    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols));
+    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols), seg);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
       uint32_t mw[2];
-      raw.bits(seg, mw);
+      raw.bits(mw);
       // mask words of the next step load while this one computes
-      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP));
+      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg);
       ok = __all_sync(0xffffffffu, mbar_wait(st_full, st & 1, ab));
       if (!ok) break;
       tc_fence_after();
@@ -726,15 +726,15 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint64_t ndl = f2_pack(-dl, -dl);
     bool ok = true;
     StepMasks<NP> raw;
-    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols));
+    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols), seg);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
       const int N = 16 * min(NP, n_cols - st * NP);
       const bool active = grp * 32 < N;
       uint32_t mw[2];
-      raw.bits(seg, mw);
+      raw.bits(mw);
       // mask words of the next step load while this one computes
-      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP));
+      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg);
       ok = __all_sync(0xffffffffu, mbar_wait(&sd_full[b], (st >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();

@@ -38,29 +38,27 @@ __device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {
   return x;
 }
 
-// The column-list mask words of one step of NP pages (16 bits per segment
-// per page).  `fetch` only issues the loads; the words are read by `bits`,
-// an iteration later, so the load latency never stalls the row math that
-// runs in between.
+// The column-list masks of one step of NP pages for one row: each entry
+// holds 16 bits per segment, and a row reads only the 16-bit half-word of
+// its own segment.  `fetch` only issues the loads; the words are read by
+// `bits`, an iteration later, so the load latency never stalls the row math
+// that runs in between.
 template <int NP>
 struct StepMasks {
-  uint64_t w[NP];
-  __device__ __forceinline__ void fetch(const uint64_t* __restrict__ masks, int first, int n) {
+  uint32_t w[NP];
+  // `seg` < 0 (a row without a segment) gives an all-zero mask.
+  __device__ __forceinline__ void fetch(const uint64_t* __restrict__ masks, int first, int n, int seg) {
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(masks + first) + (seg < 0 ? 0 : seg);
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
-      w[j] = 0ull;
-      if (j < n) w[j] = __ldg(masks + first + j);
+      w[j] = 0u;
+      if (j < n && seg >= 0) w[j] = __ldg(h + 4 * j);
     }
   }
-  // Row mask of the step: bit c of word c/32 <=> column c may be attended by
-  // a row of segment `seg`; `seg` < 0 gives an all-zero mask.
-  __device__ __forceinline__ void bits(int seg, uint32_t (&mw)[NP / 2]) const {
+  // Row mask of the step: bit c of word c/32 <=> column c may be attended.
+  __device__ __forceinline__ void bits(uint32_t (&mw)[NP / 2]) const {
 #pragma unroll
-    for (int i = 0; i < NP / 2; ++i) mw[i] = 0u;
-    if (seg < 0) return;
-#pragma unroll
-    for (int j = 0; j < NP; ++j)
-      mw[j >> 1] |= (static_cast<uint32_t>(w[j] >> (16 * seg)) & 0xFFFFu) << (16 * (j & 1));
+    for (int i = 0; i < NP / 2; ++i) mw[i] = w[2 * i] | (w[2 * i + 1] << 16);
   }
 };
 
