@@ -23,6 +23,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libspattn.so")
 
 SPATTN_OK = 0
+SPATTN_ERR_INVALID_ARG, SPATTN_ERR_UNSUPPORTED, SPATTN_ERR_OOM, SPATTN_ERR_CUDA = 1, 2, 3, 4
+SPATTN_ERR_TIMEOUT, SPATTN_ERR_DEVICE = 5, 6
 STATUS_NAMES = {
     0: "SPATTN_OK",
     1: "SPATTN_ERR_INVALID_ARG",
@@ -36,7 +38,7 @@ STATUS_NAMES = {
 ENTRY_POINTS = (
     "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_bwd_noalloc", "spattn_check", "spattn_plan_stats", "spattn_profile",
     "spattn_profile_read", "spattn_plan_pages", "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy",
-    "spattn_status_string",
+    "spattn_status_string", "spattn_wait_selftest",
 )
 
 
@@ -89,6 +91,7 @@ def _lib():
         lib.spattn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
         lib.spattn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
         lib.spattn_check.argtypes = [P, P]
+        lib.spattn_wait_selftest.argtypes = [P, I64, P]
         lib.spattn_plan_stats.argtypes = [P, ctypes.POINTER(_Stats)]
         lib.spattn_plan_pages.argtypes = [P, I32, I64, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64)]
         lib.spattn_plan_qblocks.argtypes = [P, I32, I64, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64)]
@@ -262,6 +265,13 @@ def spattn_bwd(q, k, v, o, lse, do, plan: Plan, dq=None, dk=None, dv=None, strea
 def spattn_check(plan: Plan, stream=None):
     """Synchronise the stream and raise if a kernel recorded a device-side error."""
     _check(_lib().spattn_check(plan.handle, _stream_handle(stream)), "spattn_check")
+
+
+def spattn_wait_selftest(plan: Plan, deadline_cycles: int, stream=None) -> int:
+    """Run the bounded-wait failure self-test; returns the following spattn_check status."""
+    _check(_lib().spattn_wait_selftest(plan.handle, int(deadline_cycles), _stream_handle(stream)),
+           "spattn_wait_selftest")
+    return _lib().spattn_check(plan.handle, _stream_handle(stream))
 
 
 def load_library():

@@ -227,6 +227,16 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }
 
+int spattn_wait_selftest(spattn_plan_t plan, int64_t deadline_cycles, void* stream) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  if (deadline_cycles < 10000 || deadline_cycles > 2000000000ll) return SPATTN_ERR_INVALID_ARG;
+  const int st = check_plan_device(plan);
+  if (st) return st;
+  return launch_wait_selftest(plan->d_err, deadline_cycles, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SPATTN_OK
+             : SPATTN_ERR_CUDA;
+}
+
 int spattn_check(spattn_plan_t plan, void* stream) {
   if (!plan) return SPATTN_ERR_INVALID_ARG;
   if (plan->device < 0) return SPATTN_ERR_CUDA;

@@ -55,6 +55,12 @@ cudaError_t launch_dq(int head_dim, const __nv_bfloat16* q, const TmaPages& tdo,
                       __nv_bfloat16* dq, cudaStream_t st);
 
 // K5: zero the rows of pages that hold no valid slot (and LSE = -inf).
+// One CTA whose warp 0 waits, with the given deadline, on an mbarrier that
+// nothing arrives at, and whose warp 1 waits on it with the tile kernels'
+// deadline: warp 0 times out and records SPATTN_ERR_TIMEOUT's device code in
+// `err`, warp 1 sees the CTA abort flag and gives up.  Both return.
+cudaError_t launch_wait_selftest(int* err, long long deadline_cycles, cudaStream_t st);
+
 cudaError_t launch_fill(int head_dim, const int32_t* pages, int64_t n_pages, int64_t bh, int64_t slots,
                         __nv_bfloat16* t0, __nv_bfloat16* t1, float* lse, cudaStream_t st);
 

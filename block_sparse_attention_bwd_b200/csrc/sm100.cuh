@@ -86,10 +86,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 #endif
 
 // Wait for the phase with the given parity to complete.  Returns false if the
-// CTA is aborting or the deadline passed (then the abort flag is raised).
-// The fast path is a bare try_wait; the deadline is checked on the cheap SM
-// cycle counter once every 1024 polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab) {
+// CTA is aborting or the deadline (SM cycles) passed (then the abort flag is
+// raised).  The fast path is a bare try_wait; the deadline is checked on the
+// cheap SM cycle counter once every 1024 polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Abort& ab,
+                                          long long deadline = SPATTN_WAIT_CYCLES) {
   if (mbar_try_wait(bar, parity)) return true;
   long long t0 = 0;
   for (uint32_t it = 1;; ++it) {
@@ -99,7 +100,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
       const long long now = clock64();
       if (t0 == 0) {
         t0 = now;
-      } else if (now - t0 > SPATTN_WAIT_CYCLES) {
+      } else if (now - t0 > deadline) {
         raise_abort(ab, kErrTimeout);
         return false;
       }

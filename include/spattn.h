@@ -145,6 +145,16 @@ int spattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* 
  * plan's kernels recorded: SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_DEVICE. */
 int spattn_check(spattn_plan_t plan, void* stream);
 
+/* Failure-path self-test of the device-side bounded waits (no fault, no
+ * hang).  Launches on `stream` one CTA that waits on a barrier nothing ever
+ * completes: one warp with a deadline of `deadline_cycles` SM cycles (10^4 ..
+ * 2*10^9, else SPATTN_ERR_INVALID_ARG), one with the tile kernels' deadline.
+ * The first times out and records a timeout in the plan's error word, the
+ * second sees the CTA's abort flag; both return, and the context stays
+ * usable.  The next spattn_check on the plan returns SPATTN_ERR_TIMEOUT (and
+ * clears it).  A host-only plan returns SPATTN_ERR_CUDA. */
+int spattn_wait_selftest(spattn_plan_t plan, int64_t deadline_cycles, void* stream);
+
 int spattn_plan_stats(spattn_plan_t plan, spattn_stats* stats);
 
 /* Per-kernel device timing.  While enabled, spattn_fwd / spattn_bwd record a

@@ -101,3 +101,25 @@ def test_inspection_rejects_out_of_range():
         pl.qblocks(0, 10 ** 6)
     with pytest.raises(sp.SpattnError):
         pl.work(2)
+
+
+def test_wait_selftest_argument_checks_on_host():
+    lib = sp.load_library()
+    assert lib.spattn_wait_selftest(None, 1_000_000, None) == 1
+    p = W.make_problem("tiny")
+    pl = _plan(p)
+    # deadline outside 10^4 .. 2*10^9 cycles
+    assert lib.spattn_wait_selftest(pl.handle, 10, None) == 1
+    assert lib.spattn_wait_selftest(pl.handle, 3_000_000_000, None) == 1
+    # a plan built without a GPU cannot launch anything
+    if not sp_device_available():
+        assert lib.spattn_wait_selftest(pl.handle, 1_000_000, None) == 4
+    pl.close()
+
+
+def sp_device_available():
+    try:
+        import torch
+        return torch.cuda.is_available()
+    except Exception:
+        return False
