@@ -233,6 +233,18 @@ def useful_pairs(p):
 # ----------------------------------------------------------------------------
 # arms
 # ----------------------------------------------------------------------------
+def reduce_max(values, dist, device):
+    """Element-wise max of `values` over all ranks: a multi-rank job takes as
+    long as its slowest rank.  Without a process group, the values as given."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+
+    tt = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+    return tt.tolist()
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -352,10 +364,7 @@ def run_ours(args):
     t_fwd = sum(a.elapsed_time(b) for a, b, _ in ev) / 1e3
     t_bwd = sum(b.elapsed_time(c) for _, b, c in ev) / 1e3
     t_total = t_fwd + t_bwd
-    if dist is not None:
-        tt = torch.tensor([t_total, t_fwd, t_bwd], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        t_total, t_fwd, t_bwd = tt.tolist()
+    t_total, t_fwd, t_bwd = reduce_max([t_total, t_fwd, t_bwd], dist, dev)
     sp.spattn_check(plan)
     K = args.steps
     value = 10 * D * U * world * K / t_total / 1e12
@@ -435,11 +444,7 @@ def run_ours(args):
         s_down.wait_stream(s_up)
         b.record(s_down)
         torch.cuda.synchronize()
-        te = a.elapsed_time(b) / 1e3
-        if dist is not None:
-            tt = torch.tensor([te], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            te = tt.item()
+        te = reduce_max([a.elapsed_time(b) / 1e3], dist, dev)[0]
         e2e = {"value": 10 * D * U * world * args.e2e_steps / te / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
                "pipelined": "two buffer sets, upload / kernels / download streams"}
