@@ -26,6 +26,7 @@
 #include <cmath>
 #include <cstring>
 #include <new>
+#include <thread>
 
 namespace spattn {
 
@@ -203,14 +204,52 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
 int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32_t heads, int32_t batch,
                    WorkList& wl) {
   const auto tiles = pack_tiles(own);
-  std::vector<uint64_t> acc(col.n_pages, 0);
-  std::vector<int32_t> touched;
+  // Heads are independent: each is built on its own into part[h] (worker t
+  // takes heads t, t + n, ...), then the parts are joined in head order, so
+  // the result does not depend on the number of threads.
+  std::vector<WorkList> part(heads);
+  const int n_threads = std::max(1, std::min<int>(heads, static_cast<int>(std::thread::hardware_concurrency())));
+  std::vector<char> failed(n_threads, 0);
+  auto worker = [&](int t) {
+    try {
+      std::vector<uint64_t> acc(col.n_pages, 0);
+      std::vector<int32_t> touched;
+      for (int32_t h = t; h < heads; h += n_threads) build_head(own, col, adj, h, tiles, part[h], acc, touched);
+    } catch (...) {
+      failed[t] = 1;  // an allocation failed; reported below as OOM
+    }
+  };
+  if (n_threads == 1) {
+    worker(0);
+  } else {
+    std::vector<std::thread> pool;
+    pool.reserve(n_threads);
+    for (int t = 0; t < n_threads; ++t) pool.emplace_back(worker, t);
+    for (auto& th : pool) th.join();
+  }
+  for (char f : failed)
+    if (f) return SPATTN_ERR_OOM;
+  size_t n_entries = 0;
+  for (const auto& pt : part) n_entries += pt.pages.size();
+  if (n_entries > static_cast<size_t>(INT32_MAX)) return SPATTN_ERR_UNSUPPORTED;
   wl.work.clear();
   wl.pages.clear();
   wl.masks.clear();
   wl.physical_pairs = 0;
-  for (int32_t h = 0; h < heads; ++h) build_head(own, col, adj, h, tiles, wl, acc, touched);
-  if (wl.pages.size() > static_cast<size_t>(INT32_MAX)) return SPATTN_ERR_UNSUPPORTED;
+  wl.pages.reserve(n_entries);
+  wl.masks.reserve(n_entries);
+  for (auto& pt : part) {
+    const int32_t off = static_cast<int32_t>(wl.pages.size());  // entry ranges are per part
+    for (size_t i = 0; i < pt.work.size(); i += kWorkWords) {
+      pt.work[i + 2] += off;
+      pt.work[i + 3] += off;
+    }
+    wl.work.insert(wl.work.end(), pt.work.begin(), pt.work.end());
+    wl.pages.insert(wl.pages.end(), pt.pages.begin(), pt.pages.end());
+    wl.masks.insert(wl.masks.end(), pt.masks.begin(), pt.masks.end());
+    wl.physical_pairs += pt.physical_pairs;
+    pt = WorkList();  // release the part's memory as soon as it is copied
+  }
   const int64_t per_batch = static_cast<int64_t>(wl.work.size()) / kWorkWords;
   std::vector<int32_t> all;
   all.reserve(static_cast<size_t>(per_batch) * batch * kWorkWords);
