@@ -24,6 +24,7 @@
 #include <algorithm>
 #include <chrono>
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <new>
 #include <thread>
@@ -208,7 +209,10 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   // takes heads t, t + n, ...), then the parts are joined in head order, so
   // the result does not depend on the number of threads.
   std::vector<WorkList> part(heads);
-  const int n_threads = std::max(1, std::min<int>(heads, static_cast<int>(std::thread::hardware_concurrency())));
+  // all hardware threads, unless SPATTN_PLAN_THREADS (>= 1) asks for fewer or more
+  int want = static_cast<int>(std::thread::hardware_concurrency());
+  if (const char* env = std::getenv("SPATTN_PLAN_THREADS")) want = std::max(1, std::atoi(env));
+  const int n_threads = std::max(1, std::min<int>(heads, want));
   std::vector<char> failed(n_threads, 0);
   auto worker = [&](int t) {
     try {

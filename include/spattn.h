@@ -116,6 +116,9 @@ typedef struct {
  * calls (stats, pages, qblocks, work) work and spattn_fwd / spattn_bwd /
  * spattn_check return SPATTN_ERR_CUDA. */
 int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_plan_t* out);
+/* (Heads are planned in parallel on all hardware threads; the environment
+ * variable SPATTN_PLAN_THREADS, if set to n >= 1, uses n threads instead.
+ * The plan is identical for every thread count.) */
 
 /* Forward: O and LSE for every query slot of every (batch, head). */
 int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, void* o, float* lse,

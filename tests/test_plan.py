@@ -150,3 +150,19 @@ def test_page_lists_and_counts_large_sampled(name):
             g = p.kv_group[j]
             exp = [] if g < 0 else np.nonzero((p.q_group >= 0) & A[np.where(p.q_group >= 0, p.q_group, 0), g])[0].tolist()
         assert got == exp
+
+
+@pytest.mark.parametrize("name", ["partial", "svg2"])
+def test_plan_independent_of_thread_count(name, monkeypatch):
+    p = W.with_heads(W.make_problem(name), 5)
+    plans = []
+    for threads in ("1", "7"):
+        monkeypatch.setenv("SPATTN_PLAN_THREADS", threads)
+        plans.append(sp.Plan.from_problem(p))
+    for which in (0, 1):
+        a, b = plans[0].work(which), plans[1].work(which)
+        for x, y in zip(a, b):
+            assert np.array_equal(x, y)
+    sa, sb = plans[0].stats(), plans[1].stats()
+    for k in ("useful_pairs", "physical_pairs_fwd", "physical_pairs_dkdv", "n_work_fwd", "n_entries_dkdv"):
+        assert sa[k] == sb[k], k
