@@ -119,22 +119,29 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons, n = [], None, set(), 0
         with open(self.path) as fh:
-            for line in fh:
-                parts = [x.strip() for x in line.split(",")]
-                if len(parts) < 9:
-                    continue
-                try:
-                    sm.append(float(parts[1]))
-                    mx = float(parts[2])
-                except ValueError:
-                    continue
-                n += 1
-                for name, val in zip(self.REASONS, parts[5:9]):
-                    if val.lower() == "active":
-                        reasons.add(name)
+            out = self.parse(fh)
         os.unlink(self.path)
+        return out
+
+    @classmethod
+    def parse(cls, lines):
+        """Median SM clock, max clock and the throttle reasons seen active in
+        `nvidia-smi --query-gpu=FIELDS --format=csv,noheader,nounits` lines."""
+        sm, mx, reasons, n = [], None, set(), 0
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            n += 1
+            for name, val in zip(cls.REASONS, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
         return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": n}
 

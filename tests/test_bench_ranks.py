@@ -78,3 +78,20 @@ def test_reference_arm_two_ranks_prints_one_line():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["value"] == d["value"] and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_clock_parse_reports_median_and_active_reasons():
+    b = _bench()
+    lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1700, 1965, 998.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1720, 1965, 999.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    r = b.ClockSampler.parse(lines)
+    assert r["samples"] == 3 and r["sm_mhz"] == 1720.0 and r["sm_max_mhz"] == 1965.0
+    assert r["reasons"] == ["sw_power_cap"]
+    r = b.ClockSampler.parse(["0, 1200, 1965, 500, 0x0, Active, Not Active, Active, Not Active"])
+    assert r["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    assert b.ClockSampler.parse([])["sm_mhz"] is None
