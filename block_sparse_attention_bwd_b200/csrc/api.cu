@@ -153,6 +153,13 @@ int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_p
       delete P;
     }
     return SPATTN_ERR_OOM;
+  } catch (...) {
+    // any other exception (e.g. std::system_error from the host runtime)
+    if (P) {
+      free_plan_device(P);
+      delete P;
+    }
+    return SPATTN_ERR_OOM;
   }
   *out = P;
   return SPATTN_OK;

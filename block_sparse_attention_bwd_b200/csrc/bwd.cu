@@ -2,20 +2,21 @@
 // tile, no atomics) and K4 (dQ owned per query tile, no atomics).
 //
 // Method (KPage abstract, "KPage: block-sparse attention for partially
-// occupied 3D blocks", zhuanzhiai.com, abstract paragraph): "K/V-owned page
-// packing" preserves the sparse graph in the backward pass.  Here the key
-// side packs its valid 16-row pages into 128-row owned tiles exactly as the
-// query side does in the forward pass; each key tile walks the query pages
-// that reach it (the transposed lists), so dK and dV are accumulated in TMEM
-// and written once.  dQ is computed by a second, query-owned pass over the
-// forward page lists.  The gradient formulas are the standard ones for
-// softmax attention: P = exp(S - LSE), dV = P^T dO, dP = dO V^T,
+// occupied 3D blocks", zhuanzhiai.com, abstract paragraph): the backward pass
+// keeps the sparse graph exact by letting the K/V side own its pages.  Here
+// the key side packs its valid 16-row pages into 128-row owned tiles exactly
+// as the query side does in the forward pass; each key tile walks the query
+// pages that reach it (the transposed lists), so dK and dV are accumulated
+// in TMEM and written once.  dQ is computed by a second, query-owned pass
+// over the forward page lists.  The gradient formulas are the standard ones
+// for softmax attention: P = exp(S - LSE), dV = P^T dO, dP = dO V^T,
 // dS = P * (dP - Delta), dK = scale dS^T Q, dQ = scale dS K.
 //
-// Both tile kernels use 11 warps: warp 0 is the TMA producer, warp 1
-// allocates TMEM and issues the two products of each step, warp 10 issues
-// the accumulating product, and warps 2..9 turn each step's scores into
-// P / dS, one tile row per lane, two warp groups per step (32 columns each).
+// Both tile kernels use 12 warps: warps 0 and 11 are TMA producers (one per
+// column tensor), warp 1 allocates TMEM and issues the two products of each
+// step that read the column tiles, warp 10 issues the accumulating products,
+// and warps 2..9 turn each step's scores into P / dS, one tile row per lane,
+// two warp groups per step (32 columns each).
 #include <algorithm>
 
 #include "kernels.cuh"

@@ -13,8 +13,6 @@
 // holds until the process exits.
 #include <cudaTypedefs.h>
 
-#include <mutex>
-
 #include "kernels.cuh"
 #include "plan.hpp"
 
@@ -27,24 +25,22 @@ namespace {
 
 // File-scope scratch for Delta.  In host code this name is only a host-side
 // stand-in, never a device address: kernels get the address that
-// cudaGetSymbolAddress returns for the current device.
+// cudaGetSymbolAddress returns in the calling thread's current context.
 static __device__ __align__(256) float g_delta_scratch[kNoAllocDeltaRows];
 
-constexpr int kMaxDevices = 64;
-float* g_scratch_ptr[kMaxDevices] = {};
-std::mutex g_scratch_mutex;
-
-// Device address of the scratch on the current device; looked up once per
-// device (the first call on that device), with that device current.
-int scratch_address(int dev, float** out) {
-  if (dev < 0 || dev >= kMaxDevices) return SPATTN_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mutex);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_delta_scratch) != cudaSuccess || !p) return SPATTN_ERR_CUDA;
-    g_scratch_ptr[dev] = static_cast<float*>(p);
+// Device address of the scratch in the current context.  It is looked up on
+// every call (a table lookup that allocates nothing) rather than cached: a
+// device reset, or a primary context that is released and created again,
+// loads the module anew and may place the array elsewhere, and a cached
+// address would then point at freed memory.  The first call in a context
+// also loads the library's device code there.
+int scratch_address(float** out) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_delta_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return SPATTN_ERR_CUDA;
   }
-  *out = g_scratch_ptr[dev];
+  *out = static_cast<float*>(p);
   return SPATTN_OK;
 }
 
@@ -72,7 +68,7 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
       !aligned(dk) || !aligned(dv))
     return SPATTN_ERR_INVALID_ARG;
   float* delta = nullptr;
-  int st = scratch_address(dev, &delta);
+  int st = scratch_address(&delta);
   if (st) return st;
   const int D = plan->head_dim;
   TmaPages tq, tk, tv, tdo;

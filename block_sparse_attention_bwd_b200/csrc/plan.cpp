@@ -9,8 +9,13 @@
 // passes use one tile shape on the tensor core (128 rows x up to 128
 // columns per step) and the planner decides what fills it:
 //   * an owned tile is up to 8 valid 16-row pages of the owned side (whole
-//     64-slot blocks packed in slot order, pages without a valid row left
-//     out), so partly occupied blocks share a tile instead of padding it;
+//     64-slot blocks, pages without a valid row left out), so partly
+//     occupied blocks share a tile instead of padding it.  Which blocks
+//     share a tile is decided per head: blocks whose column lists overlap
+//     most are grouped (every row of a tile runs over the union of the
+//     tile's lists), and the result is kept if it computes fewer physical
+//     pairs than plain slot order;
+//   * the work items of a head run longest column list first;
 //   * the tile's column list is the sorted union of the other side's pages
 //     reachable from the groups in the tile, each with one 16-bit row mask
 //     per group ("segment") present in the tile, so masking stays exact
@@ -26,8 +31,11 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <iterator>
 #include <new>
+#include <queue>
 #include <thread>
+#include <tuple>
 
 namespace spattn {
 
@@ -116,27 +124,190 @@ void build_bwd_adjacency(const Adjacency& f, int32_t heads, int32_t n_q, int32_t
     }
 }
 
-// Owned tiles: whole 64-slot blocks, valid pages only, packed in slot order
-// while the tile holds at most 8 pages.
-std::vector<std::vector<int32_t>> pack_tiles(const Side& s) {
-  std::vector<std::vector<int32_t>> tiles;
-  std::vector<int32_t> cur;
-  const int64_t n_blocks = (s.slots + kBlockRows - 1) / kBlockRows;
+// A 64-slot block of the owned side: its valid pages and its groups.
+struct OwnBlock {
+  int32_t pages[kBlockRows / kPageRows];
+  int npg = 0;
+  std::vector<int32_t> groups;  // distinct, ascending
+};
+
+std::vector<OwnBlock> owned_blocks(const Side& s) {
   const int per = kBlockRows / kPageRows;
+  std::vector<OwnBlock> out;
+  const int64_t n_blocks = (s.n_pages + per - 1) / per;
   for (int64_t blk = 0; blk < n_blocks; ++blk) {
-    std::vector<int32_t> vp;
+    OwnBlock b;
     for (int i = 0; i < per; ++i) {
       const int64_t p = blk * per + i;
-      if (p < s.n_pages && s.page_mask[p]) vp.push_back(static_cast<int32_t>(p));
+      if (p < s.n_pages && s.page_mask[p]) b.pages[b.npg++] = static_cast<int32_t>(p);
     }
-    if (vp.empty()) continue;
-    if (cur.size() + vp.size() > static_cast<size_t>(kTilePages)) {
+    if (b.npg == 0) continue;
+    const int64_t r1 = std::min<int64_t>((blk + 1) * per * kPageRows, s.slots);
+    for (int64_t i = blk * per * kPageRows; i < r1; ++i)
+      if (s.group[i] >= 0) b.groups.push_back(s.group[i]);
+    std::sort(b.groups.begin(), b.groups.end());
+    b.groups.erase(std::unique(b.groups.begin(), b.groups.end()), b.groups.end());
+    out.push_back(std::move(b));
+  }
+  return out;
+}
+
+// Owned tiles in slot order: whole blocks appended while the tile holds at
+// most 8 pages.
+std::vector<std::vector<int32_t>> pack_slot_order(const std::vector<OwnBlock>& blocks) {
+  std::vector<std::vector<int32_t>> tiles;
+  std::vector<int32_t> cur;
+  for (const auto& b : blocks) {
+    if (cur.size() + b.npg > static_cast<size_t>(kTilePages)) {
       tiles.push_back(cur);
       cur.clear();
     }
-    cur.insert(cur.end(), vp.begin(), vp.end());
+    cur.insert(cur.end(), b.pages, b.pages + b.npg);
   }
   if (!cur.empty()) tiles.push_back(cur);
+  return tiles;
+}
+
+size_t union_size(const std::vector<int32_t>& a, const std::vector<int32_t>& b) {
+  size_t n = 0, i = 0, j = 0;
+  while (i < a.size() && j < b.size()) {
+    if (a[i] == b[j]) { ++i; ++j; }
+    else if (a[i] < b[j]) ++i;
+    else ++j;
+    ++n;
+  }
+  return n + (a.size() - i) + (b.size() - j);
+}
+
+// Owned tiles grouped by the similarity of what their rows attend (the
+// query-side routing of the KPage abstract, B200 form): every row of a tile
+// runs over the union of the tile's column lists, so blocks whose column
+// lists overlap most are packed together.  Greedy agglomeration: the pair of
+// clusters with the largest overlap (column groups they share, weighted by
+// the pages of each group) merges first, while the merged cluster holds at
+// most 8 pages and at most 4 groups (one work item).  Clusters left with room
+// are then filled in slot order under the same limits.
+std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency& adj, int32_t h,
+                                               const std::vector<OwnBlock>& blocks) {
+  const int32_t nb = static_cast<int32_t>(blocks.size());
+  std::vector<std::vector<int32_t>> sig(nb);
+  for (int32_t b = 0; b < nb; ++b) {
+    for (int32_t g : blocks[b].groups) {
+      const int64_t r = static_cast<int64_t>(h) * adj.n_src + g;
+      sig[b].insert(sig[b].end(), adj.dst.begin() + adj.ptr[r], adj.dst.begin() + adj.ptr[r + 1]);
+    }
+    std::sort(sig[b].begin(), sig[b].end());
+    sig[b].erase(std::unique(sig[b].begin(), sig[b].end()), sig[b].end());
+  }
+  auto wt = [&](int32_t g) { return col.gp_ptr[g + 1] - col.gp_ptr[g]; };
+  // column group -> blocks whose signature holds it
+  std::vector<int64_t> ip(static_cast<size_t>(col.n_groups) + 1, 0);
+  for (int32_t b = 0; b < nb; ++b)
+    for (int32_t g : sig[b]) ip[g + 1] += 1;
+  for (int32_t g = 0; g < col.n_groups; ++g) ip[g + 1] += ip[g];
+  std::vector<int32_t> iv(ip.back());
+  {
+    std::vector<int64_t> fill(ip.begin(), ip.end() - 1);
+    for (int32_t b = 0; b < nb; ++b)
+      for (int32_t g : sig[b]) iv[fill[g]++] = b;
+  }
+  std::vector<int32_t> parent(nb), npg(nb);
+  std::vector<std::vector<int32_t>> groups(nb), members(nb);
+  for (int32_t b = 0; b < nb; ++b) {
+    parent[b] = b;
+    npg[b] = blocks[b].npg;
+    groups[b] = blocks[b].groups;
+    members[b] = {b};
+  }
+  auto find = [&](int32_t x) {
+    while (parent[x] != x) x = parent[x] = parent[parent[x]];
+    return x;
+  };
+  auto fits = [&](int32_t a, int32_t b) {
+    return npg[a] + npg[b] <= kTilePages && union_size(groups[a], groups[b]) <= static_cast<size_t>(kMaxSegments);
+  };
+  auto overlap = [&](int32_t a, int32_t b) {
+    int64_t w = 0;
+    size_t i = 0, j = 0;
+    while (i < sig[a].size() && j < sig[b].size()) {
+      if (sig[a][i] == sig[b][j]) { w += wt(sig[a][i]); ++i; ++j; }
+      else if (sig[a][i] < sig[b][j]) ++i;
+      else ++j;
+    }
+    return w;
+  };
+  // (overlap, -distance in slot order, a, b): ties go to nearby blocks
+  using Cand = std::tuple<int64_t, int32_t, int32_t, int32_t>;
+  std::priority_queue<Cand> heap;
+  std::vector<int64_t> cnt(nb, 0);
+  std::vector<int32_t> touched;
+  // Candidates of cluster a: clusters sharing a column group.  The counts are
+  // exact before any merge and upper bounds after; every popped candidate is
+  // re-evaluated exactly.
+  auto push_candidates = [&](int32_t a, bool only_greater) {
+    touched.clear();
+    for (int32_t g : sig[a])
+      for (int64_t x = ip[g]; x < ip[g + 1]; ++x) {
+        const int32_t r = find(iv[x]);
+        if (r == a || (only_greater && r < a)) continue;
+        if (cnt[r] == 0) touched.push_back(r);
+        cnt[r] += wt(g);
+      }
+    for (int32_t r : touched) {
+      if (cnt[r] > 0 && fits(a, r)) heap.emplace(cnt[r], -std::abs(r - a), std::min(a, r), std::max(a, r));
+      cnt[r] = 0;
+    }
+  };
+  for (int32_t b = 0; b < nb; ++b) push_candidates(b, true);
+  while (!heap.empty()) {
+    const auto [w, nd, a, b] = heap.top();
+    heap.pop();
+    if (parent[a] != a || parent[b] != b || !fits(a, b)) continue;
+    const int64_t exact = overlap(a, b);
+    if (exact != w) {
+      if (exact > 0) heap.emplace(exact, nd, a, b);
+      continue;
+    }
+    // merge b into a
+    parent[b] = a;
+    npg[a] += npg[b];
+    std::vector<int32_t> u;
+    std::set_union(groups[a].begin(), groups[a].end(), groups[b].begin(), groups[b].end(), std::back_inserter(u));
+    groups[a].swap(u);
+    u.clear();
+    std::set_union(sig[a].begin(), sig[a].end(), sig[b].begin(), sig[b].end(), std::back_inserter(u));
+    sig[a].swap(u);
+    std::vector<int32_t>().swap(sig[b]);
+    members[a].insert(members[a].end(), members[b].begin(), members[b].end());
+    std::vector<int32_t>().swap(members[b]);
+    if (npg[a] < kTilePages) push_candidates(a, false);
+  }
+  // fill: clusters left with room, in slot order of their first block (a
+  // cluster's root is its lowest block index)
+  std::vector<int32_t> heads_of_tiles;
+  int32_t cur = -1;
+  for (int32_t r = 0; r < nb; ++r) {
+    if (parent[r] != r) continue;
+    if (cur >= 0 && fits(cur, r)) {
+      npg[cur] += npg[r];
+      std::vector<int32_t> u;
+      std::set_union(groups[cur].begin(), groups[cur].end(), groups[r].begin(), groups[r].end(),
+                     std::back_inserter(u));
+      groups[cur].swap(u);
+      members[cur].insert(members[cur].end(), members[r].begin(), members[r].end());
+      continue;
+    }
+    cur = r;
+    heads_of_tiles.push_back(r);
+  }
+  std::vector<std::vector<int32_t>> tiles;
+  tiles.reserve(heads_of_tiles.size());
+  for (int32_t r : heads_of_tiles) {
+    std::vector<int32_t> pages;
+    for (int32_t b : members[r]) pages.insert(pages.end(), blocks[b].pages, blocks[b].pages + blocks[b].npg);
+    std::sort(pages.begin(), pages.end());
+    tiles.push_back(std::move(pages));
+  }
   return tiles;
 }
 
@@ -202,9 +373,40 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
   }
 }
 
+// Items of one head, longest column list first: CTAs start in grid order,
+// so the longest items start earliest and short ones fill in at the end.
+void order_longest_first(WorkList& w) {
+  const size_t n = w.work.size() / kWorkWords;
+  std::vector<size_t> idx(n);
+  for (size_t i = 0; i < n; ++i) idx[i] = i;
+  std::stable_sort(idx.begin(), idx.end(), [&](size_t x, size_t y) {
+    const int32_t* a = w.work.data() + x * kWorkWords;
+    const int32_t* b = w.work.data() + y * kWorkWords;
+    return (a[3] - a[2]) > (b[3] - b[2]);
+  });
+  std::vector<int32_t> out;
+  out.reserve(w.work.size());
+  for (size_t i : idx) out.insert(out.end(), w.work.begin() + i * kWorkWords, w.work.begin() + (i + 1) * kWorkWords);
+  w.work.swap(out);
+}
+
+// Tile packing of a pass: 0 = best of the two per head (default), 1 = slot
+// order only, 2 = similarity grouping only.  SPATTN_PLAN_PACK=slot|similar
+// selects one (for comparisons and tests).
+int packing_mode() {
+  const char* env = std::getenv("SPATTN_PLAN_PACK");
+  if (!env) return 0;
+  if (std::strcmp(env, "slot") == 0) return 1;
+  if (std::strcmp(env, "similar") == 0) return 2;
+  return 0;
+}
+
 int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32_t heads, int32_t batch,
                    WorkList& wl) {
-  const auto tiles = pack_tiles(own);
+  const auto blocks = owned_blocks(own);
+  const auto slot_tiles = pack_slot_order(blocks);
+
+  const int mode = packing_mode();
   // Heads are independent: each is built on its own into part[h] (worker t
   // takes heads t, t + n, ...), then the parts are joined in head order, so
   // the result does not depend on the number of threads.
@@ -218,7 +420,18 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
     try {
       std::vector<uint64_t> acc(col.n_pages, 0);
       std::vector<int32_t> touched;
-      for (int32_t h = t; h < heads; h += n_threads) build_head(own, col, adj, h, tiles, part[h], acc, touched);
+      for (int32_t h = t; h < heads; h += n_threads) {
+        // Per head, the packing with fewer physical pairs (then fewer items).
+        if (mode != 2) build_head(own, col, adj, h, slot_tiles, part[h], acc, touched);
+        if (mode != 1) {
+          WorkList sim;
+          build_head(own, col, adj, h, pack_similar(col, adj, h, blocks), sim, acc, touched);
+          const bool better = mode == 2 || sim.physical_pairs < part[h].physical_pairs ||
+                              (sim.physical_pairs == part[h].physical_pairs && sim.work.size() < part[h].work.size());
+          if (better) part[h] = std::move(sim);
+        }
+        order_longest_first(part[h]);
+      }
     } catch (...) {
       failed[t] = 1;  // an allocation failed; reported below as OOM
     }
@@ -226,9 +439,17 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   if (n_threads == 1) {
     worker(0);
   } else {
+    // A thread that cannot be created (std::system_error, or bad_alloc for
+    // the pool) leaves its share to the calling thread; threads already
+    // started are always joined, so nothing escapes the C ABI.
     std::vector<std::thread> pool;
-    pool.reserve(n_threads);
-    for (int t = 0; t < n_threads; ++t) pool.emplace_back(worker, t);
+    int started = 0;
+    try {
+      pool.reserve(n_threads);
+      for (; started < n_threads; ++started) pool.emplace_back(worker, started);
+    } catch (...) {
+    }
+    for (int t = started; t < n_threads; ++t) worker(t);
     for (auto& th : pool) th.join();
   }
   for (char f : failed)

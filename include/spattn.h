@@ -55,7 +55,7 @@ enum spattn_status {
   SPATTN_OK = 0,
   SPATTN_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad group id */
   SPATTN_ERR_UNSUPPORTED = 2, /* head_dim not 64/128, slots beyond int32 rows, ... */
-  SPATTN_ERR_OOM = 3,         /* host or device allocation failed in spattn_plan */
+  SPATTN_ERR_OOM = 3,         /* spattn_plan ran out of host or device memory (or host threads) */
   SPATTN_ERR_CUDA = 4,        /* a CUDA runtime call failed */
   SPATTN_ERR_TIMEOUT = 5,     /* a kernel gave up on a device-side wait */
   SPATTN_ERR_DEVICE = 6       /* a kernel rejected its work item */
@@ -109,7 +109,12 @@ typedef struct {
 
 /* Build a plan: validate layout and graph, find valid 16-row pages, pack
  * owned tiles, and build the per-tile page lists and masks for the forward /
- * dQ pass (query-owned) and the dK/dV pass (key-owned).  Host arrays are
+ * dQ pass (query-owned) and the dK/dV pass (key-owned).
+ * Source: the KPage abstract (zhuanzhiai.com paper page), which packs
+ * 16-row K/V pages holding valid rows into large tiles across logical-block
+ * boundaries, chooses tile shapes for query blocks so that less query-side
+ * padding is computed, and has the K/V side own its pages in the backward
+ * pass.  Host arrays are
  * copied and may be freed afterwards.  Device lists are allocated on the
  * current device with cudaMalloc and owned by the plan.  On a machine with no
  * usable CUDA device the plan is built on the host only: the inspection
@@ -118,14 +123,26 @@ typedef struct {
 int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_plan_t* out);
 /* (Heads are planned in parallel on all hardware threads; the environment
  * variable SPATTN_PLAN_THREADS, if set to n >= 1, uses n threads instead.
- * The plan is identical for every thread count.) */
+ * The plan is identical for every thread count.  Per head and pass, the
+ * planner groups 64-slot blocks into owned tiles in two ways, slot order and
+ * grouping by the overlap of the blocks' column lists, and keeps the one
+ * that computes fewer physical pairs; SPATTN_PLAN_PACK=slot or =similar
+ * forces one of them.  Work items of a head run longest column list
+ * first.) */
 
-/* Forward: O and LSE for every query slot of every (batch, head). */
+/* Forward: O and LSE for every query slot of every (batch, head): masked
+ * softmax attention over exactly the plan's sparse graph, computed over the
+ * packed pages; the KPage abstract (zhuanzhiai.com paper page) states that
+ * exact masking keeps the original graph intact in the forward pass. */
 int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, void* o, float* lse,
                void* stream);
 
 /* Backward: dQ, dK, dV given O and LSE from spattn_fwd and the loss
- * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O). */
+ * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O).
+ * dK and dV are accumulated per owned key tile and written once, with no
+ * atomics: the KPage abstract (zhuanzhiai.com paper page) keeps the graph
+ * exact in the backward pass by letting the K/V side own its pages.  The
+ * gradient formulas are those of softmax attention. */
 int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* d_o,
                spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream);
 
@@ -136,16 +153,19 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
  * arguments and results.  Its fp32 scratch (one value per query row) is a
  * fixed static device array of 4,194,304 floats (16 MiB) that every GPU
  * loading the library holds until exit, so batch * heads * q_slots must not
- * exceed 4,194,304 (else SPATTN_ERR_UNSUPPORTED, nothing launched).  The
- * first call on each device performs a one-time set-up (it looks up the
- * array's device address) and should come before any stream capture.  All
+ * exceed 4,194,304 (else SPATTN_ERR_UNSUPPORTED, nothing launched).  Each
+ * call looks up the array's device address in the current context (no
+ * allocation; a device reset therefore cannot leave a stale address), and
+ * the first call on each device also loads the library's device code there,
+ * so that first call should come before any stream capture.  All
  * calls share the array and every call rewrites what it reads, so calls that
  * overlap on the GPU (on different streams) race with each other. */
 int spattn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                        const void* d_o, spattn_plan_t plan, void* dq, void* dk, void* dv, void* stream);
 
 /* Synchronise `stream` and report (then clear) any device-side error the
- * plan's kernels recorded: SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_DEVICE. */
+ * plan's kernels recorded: SPATTN_OK, SPATTN_ERR_TIMEOUT or SPATTN_ERR_DEVICE.
+ * (Failure reporting; the paper has no counterpart.) */
 int spattn_check(spattn_plan_t plan, void* stream);
 
 /* Failure-path self-test of the device-side bounded waits (no fault, no
@@ -158,9 +178,15 @@ int spattn_check(spattn_plan_t plan, void* stream);
  * clears it).  A host-only plan returns SPATTN_ERR_CUDA. */
 int spattn_wait_selftest(spattn_plan_t plan, int64_t deadline_cycles, void* stream);
 
+/* Pair accounting of the plan: useful pairs (allowed query-key pairs) and
+ * the physical pairs each pass computes, the two counts the KPage abstract
+ * (zhuanzhiai.com paper page) compares for its aggregate result, plus the
+ * 64x64 block count of a BSA-style kernel for reference.  Fills *stats;
+ * never launches. */
 int spattn_plan_stats(spattn_plan_t plan, spattn_stats* stats);
 
-/* Per-kernel device timing.  While enabled, spattn_fwd / spattn_bwd record a
+/* Per-kernel device timing, for kernel-only measurements like the forward
+ * kernel timings the KPage abstract reports (zhuanzhiai.com paper page).  While enabled, spattn_fwd / spattn_bwd record a
  * CUDA event pair around every kernel they launch, on the launch stream.
  * spattn_profile(plan, 1) starts recording, (plan, 0) stops; both discard
  * what was recorded.  spattn_profile_read waits for the recorded events,
@@ -169,15 +195,18 @@ int spattn_profile(spattn_plan_t plan, int enable);
 int spattn_profile_read(spattn_plan_t plan, spattn_kernel_times* out);
 
 /* Canonical page list of (head, Q block): ascending pages holding at least
- * one key that some query of the block may attend.  *pages points into a
+ * one key that some query of the block may attend (the 16-row K/V pages a Q
+ * block needs; KPage abstract, zhuanzhiai.com paper page).  *pages points into a
  * plan-owned buffer that stays valid until the next call on this plan. */
 int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const int32_t** pages, int64_t* n);
 
 /* Transposed list of (head, page): ascending Q blocks whose canonical list
- * holds the page.  Same buffer rules as spattn_plan_pages. */
+ * holds the page (what a key-owned backward tile walks; KPage abstract,
+ * zhuanzhiai.com paper page).  Same buffer rules as spattn_plan_pages. */
 int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const int32_t** qblocks, int64_t* n);
 
-/* Host copy of a work list, for inspection and tests.  which = 0: query-owned
+/* Host copy of a work list, for inspection and tests (the packed tiles of
+ * the KPage abstract's load-time packing, zhuanzhiai.com paper page).  which = 0: query-owned
  * (forward and dQ), 1: key-owned (dK/dV).  Each work item is 32 int32 words:
  *   [0] batch*heads + head   [1] owned page count n (<= 8)
  *   [2] first entry          [3] end entry (into pages/masks)
@@ -190,8 +219,13 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
 int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work,
                      const int32_t** pages, const uint64_t** masks, int64_t* n_entries);
 
+/* Free the plan and its device lists (NULL is a no-op).  The caller must
+ * make sure no kernel launched with the plan is still running.  (Plan
+ * lifetime; the paper has no counterpart.) */
 void spattn_plan_destroy(spattn_plan_t plan);
 
+/* Static English text of a status code; never NULL.  (Error reporting; the
+ * paper has no counterpart.) */
 const char* spattn_status_string(int status);
 
 #ifdef __cplusplus

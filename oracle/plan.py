@@ -2,9 +2,9 @@
 
 Test infrastructure only (see the package docstring).  Source: the KPage
 abstract ("KPage: block-sparse attention for partially occupied 3D blocks",
-zhuanzhiai.com, abstract paragraph): K/V are handled as "valid 16-row
-pages", and its accounting contrasts physical query-key pair capacity with
-useful interactions.
+zhuanzhiai.com, abstract paragraph): K/V are handled as 16-row pages that
+hold at least one valid row, and its accounting sets the physical query-key
+pair capacity of the tiles against the useful (allowed) pairs.
 
 Definitions (readings stated where the pages are silent):
 

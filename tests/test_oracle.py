@@ -318,3 +318,41 @@ def test_sta_useful_pairs_separable_closed_form(name, grid, window, heads):
     assert got == expect
     if name == "full":
         assert got == 16 * 256 * 64 * 27 * 64
+
+
+def test_sparse_counts_by_hand():
+    """A sparse three-block case counted by hand (BSA block pairs, useful pairs, page lists).
+
+    Query slots (3 blocks of 64): block 0 = group 0 except slot 60 = group 2;
+    block 1 = group 1; block 2 padded except slot 130 = group 2.
+    Key slots (3 blocks of 64): block 0 = group 0; block 1 padded except
+    slot 100 = group 1; block 2 = group 2.
+    Graph: q0 -> {k1}, q1 -> {} (attends nothing), q2 -> {k0, k2}.
+
+    Block pairs with an allowed pair: Q block 0 reaches K blocks 1 (via q0 ->
+    slot 100) and 0, 2 (via slot 60 -> k0, k2); Q block 1 none; Q block 2
+    reaches K blocks 0 and 2: five pairs.  Counting every pair of blocks that
+    merely hold valid slots would give 9, counting allowed group pairs 3.
+    Useful pairs: 63 * 1 (q0 -> k1) + 2 * (64 + 64) (q2 -> k0, k2) = 319.
+    """
+    qg = np.zeros(192, np.int32)
+    qg[60] = 2
+    qg[64:128] = 1
+    qg[128:] = -1
+    qg[130] = 2
+    kg = np.zeros(192, np.int32)
+    kg[64:128] = -1
+    kg[100] = 1
+    kg[128:] = 2
+    row_ptr = np.array([0, 1, 1, 3], np.int64)
+    cols = np.array([1, 0, 2], np.int32)
+    A = oracle.allowed_groups(row_ptr, cols, 3, 3, 0)
+    assert oracle.bsa_physical_pairs(qg, kg, A) == 5 * 64 * 64
+    assert oracle.useful_pairs_bruteforce(qg, kg, A) == 319
+    assert oracle.useful_pairs_closed_form(qg, kg, row_ptr, cols, 3, 3, 1) == 319
+    assert oracle.canonical_pages(qg, kg, A, 0).tolist() == [0, 1, 2, 3, 6, 8, 9, 10, 11]
+    assert oracle.canonical_pages(qg, kg, A, 1).tolist() == []
+    assert oracle.canonical_pages(qg, kg, A, 2).tolist() == [0, 1, 2, 3, 8, 9, 10, 11]
+    assert oracle.transposed_qblocks(qg, kg, A, 6).tolist() == [0]
+    assert oracle.transposed_qblocks(qg, kg, A, 4).tolist() == []
+    assert oracle.transposed_qblocks(qg, kg, A, 9).tolist() == [0, 2]

@@ -3,10 +3,12 @@
 Callers that cannot allocate device memory when they run the backward pass
 (another allocator owns the GPU, or a fixed memory budget) use this entry
 point; its scratch is a static device array inside the library.  These tests
-call it through the C ABI twice in a row and compare each result with
-spattn_bwd (same tolerance as the parity tests: relative L2 <= 1e-2 over
-valid rows; padded rows must be exact zeros), and check that sizes beyond
-the static scratch are rejected before anything is launched.
+call it through the C ABI twice in a row, the second time with a different
+dO, and compare each result with spattn_bwd on the same inputs.  Both paths
+run the same deterministic, atomic-free kernels, so the outputs must be
+bit-identical; the second call would differ if it read the first call's
+Delta from the shared scratch instead of rewriting it.  Sizes beyond the
+static scratch must be rejected before anything is launched.
 
 This file is collected last on purpose, so that a run stopping at the first
 failure has already run every other test.
@@ -26,35 +28,31 @@ pytestmark = pytest.mark.gpu
 SCRATCH_ROWS = 1 << 22
 
 
-def _rel_l2(a, b):
-    a = a.double()
-    b = b.double()
-    return float((a - b).norm() / max(float(b.norm()), 1e-30))
-
-
 @pytest.mark.parametrize("name", ["tiny_svg2", "tiny_d128", "tiny_vsa"])
 def test_noalloc_matches_bwd_on_two_calls(name):
     p = W.make_problem(name)
     t = {k: v.cuda() for k, v in W.make_tensors(p).items()}
     plan = sp.Plan.from_problem(p)
     o, lse = sp.spattn_fwd(t["q"], t["k"], t["v"], plan)
-    ref = sp.spattn_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], plan)
-    sp.spattn_check(plan)
+    # a second loss gradient: another seeded draw, same shape (padded rows keep the sentinel)
+    do2 = torch.flip(t["do"], dims=[3]).contiguous() * 0.5
     lib = sp.load_library()
     stream = torch.cuda.current_stream()
-    vq = torch.from_numpy(p.q_group >= 0).cuda()
-    vk = torch.from_numpy(p.kv_group >= 0).cuda()
-    for _call in range(2):
+    for do in (t["do"], do2):
+        ref = sp.spattn_bwd(t["q"], t["k"], t["v"], o, lse, do, plan)
+        sp.spattn_check(plan)
         # pre-fill with a value the pass must overwrite everywhere
         out = [torch.full_like(r, 7.0) for r in ref]
-        st = lib.spattn_bwd_noalloc(*(ctypes.c_void_p(x.data_ptr()) for x in (t["q"], t["k"], t["v"], o, lse, t["do"])),
+        st = lib.spattn_bwd_noalloc(*(ctypes.c_void_p(x.data_ptr()) for x in (t["q"], t["k"], t["v"], o, lse, do)),
                                     plan.handle, *(ctypes.c_void_p(x.data_ptr()) for x in out),
                                     ctypes.c_void_p(stream.cuda_stream))
         assert st == 0, sp.STATUS_NAMES.get(st, st)
         sp.spattn_check(plan)
-        for got, want, valid in zip(out, ref, (vq, vk, vk)):
-            assert _rel_l2(got[:, :, valid], want[:, :, valid]) <= 1e-2
-            assert torch.all(got[:, :, ~valid] == 0)
+        for got, want in zip(out, ref):
+            assert torch.equal(got, want)
+    # the two calls really saw different gradients
+    assert not torch.equal(sp.spattn_bwd(t["q"], t["k"], t["v"], o, lse, do2, plan)[0],
+                           sp.spattn_bwd(t["q"], t["k"], t["v"], o, lse, t["do"], plan)[0])
 
 
 def test_noalloc_rejects_rows_beyond_scratch():

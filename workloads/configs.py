@@ -57,7 +57,7 @@ import numpy as np
 PAD_SENTINEL = 1000.0
 
 CONFIG_NAMES = ("tiny", "full", "partial", "vsa", "svg2")
-EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey")
+EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_nokeys")
 
 
 @dataclasses.dataclass
@@ -243,6 +243,16 @@ def make_problem(name: str) -> Problem:
         row_ptr, cols = _csr([[0], [0, 1]])
         return Problem(name, 1, 1, 64, qg, kg, 2, 2, row_ptr, cols, 14000,
                        "ragged 40x50 slots; query group 0 attends a single key")
+    if name == "tiny_nokeys":
+        # head 0: a clamped 1x1x3 window; head 1: no query attends anything, so
+        # every work item of that head has an empty column list (and every key
+        # tile of that head receives no gradient)
+        group, tiles = sta_layout((5, 6, 10))
+        rp, cols = sta_graph(tiles, (1, 1, 3), 1)
+        rows = [cols[rp[a]:rp[a + 1]].tolist() for a in range(12)] + [[] for _ in range(12)]
+        row_ptr, cols = _csr(rows)
+        return Problem(name, 1, 2, 64, group, group.copy(), 12, 12, row_ptr, cols, 15000,
+                       "tiny STA; head 1 attends nothing (empty column lists)")
     raise KeyError(name)
 
 
