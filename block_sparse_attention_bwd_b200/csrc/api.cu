@@ -66,7 +66,27 @@ bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, 
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 5D view of strided pages: (64 columns, 4 rows, 4 groups 16 rows apart,
+// slot, batch*head).  The row and group dimensions overlap the slot
+// dimension; every box the kernels request lies inside one (batch, head),
+// because the planner only forms a strided page when all 16 of its slots
+// exist.
+bool make_strided_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(head_dim) * 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(head_dim), 4, 4, static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[4] = {row_bytes, 16 * row_bytes, row_bytes, row_bytes * static_cast<cuuint64_t>(rows)};
+  cuuint32_t box[5] = {64, 4, 4, 1, 1};
+  cuuint32_t es[5] = {1, 1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+  if (!make_strided_map(&t->m4s, ptr, head_dim, rows, bh)) return false;
   if (!make_map(&t->m16, ptr, head_dim, rows, bh, 16) || !make_map(&t->m32, ptr, head_dim, rows, bh, 32) ||
       !make_map(&t->m64, ptr, head_dim, rows, bh, 64))
     return false;
@@ -104,7 +124,7 @@ cudaError_t timed(spattn_plan_s* P, int kernel, cudaStream_t s, F&& launch) {
   return e;
 }
 
-int64_t fill_launches(const std::vector<int32_t>& pages) { return pages.empty() ? 0 : 1; }
+int64_t fill_launches(const std::vector<int32_t>& fill) { return fill.empty() ? 0 : 1; }
 
 TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots, int64_t col_slots) {
   TileArgs a;
@@ -181,10 +201,10 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
   cudaError_t e = timed(plan, SPATTN_K_FWD, s, [&] {
     return launch_fwd(D, tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), O, lse, s);
   });
-  if (e == cudaSuccess && !plan->q_invalid_pages.empty())
+  if (e == cudaSuccess && !plan->q_fill.empty())
     e = timed(plan, SPATTN_K_FILL, s, [&] {
-      return launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots,
-                         O, nullptr, lse, s);
+      return launch_fill(D, plan->d_q_fill, static_cast<int64_t>(plan->q_fill.size() / 2), bh, plan->q.slots, O,
+                         nullptr, lse, s);
     });
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }
@@ -221,15 +241,15 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
       return launch_dq(D, static_cast<const __nv_bfloat16*>(q), tdo, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse,
                        plan->d_delta, dQ, s);
     });
-  if (e == cudaSuccess && !plan->k_invalid_pages.empty())
+  if (e == cudaSuccess && !plan->k_fill.empty())
     e = timed(plan, SPATTN_K_FILL, s, [&] {
-      return launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots,
-                         dK, dV, nullptr, s);
+      return launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh, plan->k.slots, dK,
+                         dV, nullptr, s);
     });
-  if (e == cudaSuccess && !plan->q_invalid_pages.empty())
+  if (e == cudaSuccess && !plan->q_fill.empty())
     e = timed(plan, SPATTN_K_FILL, s, [&] {
-      return launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots,
-                         dQ, nullptr, nullptr, s);
+      return launch_fill(D, plan->d_q_fill, static_cast<int64_t>(plan->q_fill.size() / 2), bh, plan->q.slots, dQ,
+                         nullptr, nullptr, s);
     });
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }
@@ -269,9 +289,9 @@ int spattn_plan_stats(spattn_plan_t plan, spattn_stats* s) {
   s->n_entries_fwd = static_cast<int64_t>(plan->wq.pages.size());
   s->n_entries_dkdv = static_cast<int64_t>(plan->wk.pages.size());
   s->device_bytes = plan->device_bytes;
-  s->launches_fwd = (plan->wq.n_work > 0) + fill_launches(plan->q_invalid_pages);
-  s->launches_bwd = 1 + (plan->wk.n_work > 0) + (plan->wq.n_work > 0) + fill_launches(plan->k_invalid_pages) +
-                    fill_launches(plan->q_invalid_pages);
+  s->launches_fwd = (plan->wq.n_work > 0) + fill_launches(plan->q_fill);
+  s->launches_bwd = 1 + (plan->wk.n_work > 0) + (plan->wq.n_work > 0) + fill_launches(plan->k_fill) +
+                    fill_launches(plan->q_fill);
   s->plan_ms = plan->plan_ms;
   return SPATTN_OK;
 }

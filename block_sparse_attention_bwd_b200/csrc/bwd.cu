@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       for (int h = 0; h < NH; ++h) {
         const int idx = lane + 32 * h;  // column of the stage
         const int pg = __shfl_sync(0xffffffffu, pg_lane, idx >> 4);
-        const int64_t slot = static_cast<int64_t>(pg) * 16 + (idx & 15);
+        const int64_t slot = pref_slot(pg, idx & 15);
         const bool ok = t < n_stages && (idx >> 4) < n_t && slot < q_slots;
         x[h] = __ldg(terms + static_cast<int64_t>(wk.bh) * q_slots + (ok ? slot : 0));
         live |= ok ? (1u << h) : 0u;
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     if (ok) {
       // group 0 writes dV, group 1 writes scale * dK
       const bool owned = code != 15u && row < 16 * wk.n_own;
-      const int64_t slot = owned ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+      const int64_t slot = owned ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
       const bool write = owned && slot < kv_slots;
       const int64_t base = (static_cast<int64_t>(wk.bh) * kv_slots + slot) * D;
       const uint32_t tacc = grp == 0 ? tDV : tDK;
@@ -689,7 +689,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint32_t code = wk.row_code(row);
     const int seg = code < 4 ? static_cast<int>(code) : -1;
     const bool owned = code != 15u && row < 16 * wk.n_own;
-    const int64_t slot = row < 16 * wk.n_own ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+    const int64_t slot = row < 16 * wk.n_own ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
     const bool loaded = row < 16 * wk.n_own && slot < q_slots;
     const bool valid_slot = owned && slot < q_slots;
     const int64_t roff = static_cast<int64_t>(wk.bh) * q_slots + slot;

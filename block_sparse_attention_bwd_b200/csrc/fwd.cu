@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     }
     if (ok) {
       const bool owned = code != 15u && row < 16 * wk.n_own;
-      const int64_t slot = owned ? static_cast<int64_t>(wk.own_page(row >> 4)) * 16 + (row & 15) : 0;
+      const int64_t slot = owned ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
       const bool write = owned && slot < q_slots;
       const bool empty = !(l > 0.f);
       const float inv = empty ? 0.f : 1.0f / l;
@@ -334,23 +334,25 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   }
 }
 
-// Zero 16-row pages that hold no valid slot; LSE rows (if given) get -inf.
-__global__ void fill_kernel(const int32_t* __restrict__ pages, int64_t n_bh, int64_t slots, int head_dim,
+// Zero the rows that no work item writes: entry e of `fill` is a page and a
+// 16-bit row mask; LSE rows (if given) get -inf.
+__global__ void fill_kernel(const int32_t* __restrict__ fill, int64_t n_bh, int64_t slots, int head_dim,
                             __nv_bfloat16* __restrict__ t0, __nv_bfloat16* __restrict__ t1, float* __restrict__ lse) {
-  const int64_t page = pages[blockIdx.x];
+  const int64_t page = fill[2 * blockIdx.x];
+  const uint32_t rows = static_cast<uint32_t>(fill[2 * blockIdx.x + 1]);
   const int vec_per_row = head_dim / 8;  // 16-byte vectors
   for (int64_t bh = blockIdx.y; bh < n_bh; bh += gridDim.y) {
     for (int i = threadIdx.x; i < 16 * vec_per_row; i += blockDim.x) {
       const int r = i / vec_per_row, c = i % vec_per_row;
       const int64_t slot = page * 16 + r;
-      if (slot >= slots) continue;
+      if (slot >= slots || !((rows >> r) & 1u)) continue;
       const int64_t off = (bh * slots + slot) * head_dim + c * 8;
       if (t0) *reinterpret_cast<uint4*>(t0 + off) = make_uint4(0, 0, 0, 0);
       if (t1) *reinterpret_cast<uint4*>(t1 + off) = make_uint4(0, 0, 0, 0);
     }
     if (lse && threadIdx.x < 16) {
       const int64_t slot = page * 16 + threadIdx.x;
-      if (slot < slots) lse[bh * slots + slot] = -INFINITY;
+      if (slot < slots && ((rows >> threadIdx.x) & 1u)) lse[bh * slots + slot] = -INFINITY;
     }
   }
 }
@@ -374,11 +376,11 @@ cudaError_t launch_fwd(int head_dim, const TmaPages& tq, const TmaPages& tk, con
   return head_dim == 128 ? launch_fwd_t<128>(tq, tk, tv, a, o, lse, st) : launch_fwd_t<64>(tq, tk, tv, a, o, lse, st);
 }
 
-cudaError_t launch_fill(int head_dim, const int32_t* pages, int64_t n_pages, int64_t bh, int64_t slots,
+cudaError_t launch_fill(int head_dim, const int32_t* fill, int64_t n, int64_t bh, int64_t slots,
                         __nv_bfloat16* t0, __nv_bfloat16* t1, float* lse, cudaStream_t st) {
-  if (n_pages == 0 || bh == 0) return cudaSuccess;
-  dim3 grid(static_cast<unsigned>(n_pages), static_cast<unsigned>(bh < 65535 ? bh : 65535));
-  fill_kernel<<<grid, 128, 0, st>>>(pages, bh, slots, head_dim, t0, t1, lse);
+  if (n == 0 || bh == 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>(n), static_cast<unsigned>(bh < 65535 ? bh : 65535));
+  fill_kernel<<<grid, 128, 0, st>>>(fill, bh, slots, head_dim, t0, t1, lse);
   return cudaGetLastError();
 }
 

@@ -22,6 +22,11 @@ struct TmaPages {
   // The same 4D view with 128-row boxes: a whole 128-row stage or owned tile
   // (chunks 16 KB apart) in one request.
   CUtensorMap m128w;
+  // Strided pages: a 5D view (64-column x, 4 rows, 4 groups 16 rows apart,
+  // slot, batch*head) whose 64 x 4 x 4 box is the 16 rows of a strided page
+  // (base slot b: rows b + 16j + r), one 64-column chunk per request; it lands
+  // as a 16-row page of that chunk.
+  CUtensorMap m4s;
 };
 
 // Everything one attention launch needs besides its tensor maps.
@@ -54,14 +59,17 @@ cudaError_t launch_dq(int head_dim, const __nv_bfloat16* q, const TmaPages& tdo,
                       const TmaPages& tv, const TileArgs& a, const float* lse, const float* delta,
                       __nv_bfloat16* dq, cudaStream_t st);
 
-// K5: zero the rows of pages that hold no valid slot (and LSE = -inf).
+// K5: zero the rows that no work item writes (and LSE = -inf).
 // One CTA whose warp 0 waits, with the given deadline, on an mbarrier that
 // nothing arrives at, and whose warp 1 waits on it with the tile kernels'
 // deadline: warp 0 times out and records SPATTN_ERR_TIMEOUT's device code in
 // `err`, warp 1 sees the CTA abort flag and gives up.  Both return.
 cudaError_t launch_wait_selftest(int* err, long long deadline_cycles, cudaStream_t st);
 
-cudaError_t launch_fill(int head_dim, const int32_t* pages, int64_t n_pages, int64_t bh, int64_t slots,
+// `fill` holds n (page, 16-bit row mask) pairs: the rows r of page p with bit r
+// set are zeroed in t0 and t1 (if given) and get LSE = -inf (if given), for
+// every (batch, head).
+cudaError_t launch_fill(int head_dim, const int32_t* fill, int64_t n, int64_t bh, int64_t slots,
                         __nv_bfloat16* t0, __nv_bfloat16* t1, float* lse, cudaStream_t st);
 
 }  // namespace spattn

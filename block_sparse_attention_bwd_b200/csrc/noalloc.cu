@@ -88,11 +88,11 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
                     dV, s);
   if (e == cudaSuccess)
     e = launch_dq(D, static_cast<const __nv_bfloat16*>(q), tdo, tk, tv, make_tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, delta, dQ, s);
-  if (e == cudaSuccess && !plan->k_invalid_pages.empty())
-    e = launch_fill(D, plan->d_k_invalid, static_cast<int64_t>(plan->k_invalid_pages.size()), bh, plan->k.slots, dK,
-                    dV, nullptr, s);
-  if (e == cudaSuccess && !plan->q_invalid_pages.empty())
-    e = launch_fill(D, plan->d_q_invalid, static_cast<int64_t>(plan->q_invalid_pages.size()), bh, plan->q.slots, dQ,
+  if (e == cudaSuccess && !plan->k_fill.empty())
+    e = launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh, plan->k.slots, dK, dV,
+                    nullptr, s);
+  if (e == cudaSuccess && !plan->q_fill.empty())
+    e = launch_fill(D, plan->d_q_fill, static_cast<int64_t>(plan->q_fill.size() / 2), bh, plan->q.slots, dQ,
                     nullptr, nullptr, s);
   return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
 }

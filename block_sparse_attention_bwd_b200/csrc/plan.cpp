@@ -124,15 +124,33 @@ void build_bwd_adjacency(const Adjacency& f, int32_t heads, int32_t n_q, int32_t
     }
 }
 
-// A 64-slot block of the owned side: its valid pages and its groups.
+// The 4-row group k that holds every set bit of a 16-bit row mask, or -1
+// (an empty mask, or rows in more than one group).
+int sub_group(uint32_t m) {
+  for (int k = 0; k < 4; ++k)
+    if (m != 0u && (m & ~(0xFu << (4 * k))) == 0u) return k;
+  return -1;
+}
+
+// Strided pages are used unless SPATTN_PLAN_STRIDED=0 (for comparisons).
+bool strided_enabled() {
+  const char* env = std::getenv("SPATTN_PLAN_STRIDED");
+  return !(env && env[0] == '0');
+}
+
+// A 64-slot block of the owned side: references to its valid pages (one
+// strided page when all four pages are valid and their valid rows share a
+// 4-row group k; the block's other rows are then padded) and its groups.
 struct OwnBlock {
   int32_t pages[kBlockRows / kPageRows];
   int npg = 0;
+  int strided_group = -1;  // k of the strided page, else -1
   std::vector<int32_t> groups;  // distinct, ascending
 };
 
 std::vector<OwnBlock> owned_blocks(const Side& s) {
   const int per = kBlockRows / kPageRows;
+  const bool strided = strided_enabled();
   std::vector<OwnBlock> out;
   const int64_t n_blocks = (s.n_pages + per - 1) / per;
   for (int64_t blk = 0; blk < n_blocks; ++blk) {
@@ -142,6 +160,17 @@ std::vector<OwnBlock> owned_blocks(const Side& s) {
       if (p < s.n_pages && s.page_mask[p]) b.pages[b.npg++] = static_cast<int32_t>(p);
     }
     if (b.npg == 0) continue;
+    if (strided && b.npg == per) {
+      const int k = sub_group(s.page_mask[b.pages[0]]);
+      bool same = k >= 0;
+      for (int i = 1; i < per && same; ++i) same = sub_group(s.page_mask[b.pages[i]]) == k;
+      const int64_t p0 = blk * per;
+      if (same && 16 * (p0 + 3) + 4 * k + 4 <= s.slots) {
+        b.pages[0] = ~static_cast<int32_t>(16 * p0 + 4 * k);
+        b.npg = 1;
+        b.strided_group = k;
+      }
+    }
     const int64_t r1 = std::min<int64_t>((blk + 1) * per * kPageRows, s.slots);
     for (int64_t i = blk * per * kPageRows; i < r1; ++i)
       if (s.group[i] >= 0) b.groups.push_back(s.group[i]);
@@ -315,6 +344,7 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
 void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t h,
                 const std::vector<std::vector<int32_t>>& tiles, WorkList& wl, std::vector<uint64_t>& acc,
                 std::vector<int32_t>& touched) {
+  const bool strided = strided_enabled();
   int32_t rg[kTilePages * kPageRows];
   for (const auto& tile : tiles) {
     const int npg = static_cast<int>(tile.size());
@@ -322,7 +352,7 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
     for (int r = 0; r < kTilePages * kPageRows; ++r) {
       int32_t g = -2;  // row does not exist in this tile / tensor
       if (r < npg * kPageRows) {
-        const int64_t slot = static_cast<int64_t>(tile[r / kPageRows]) * kPageRows + r % kPageRows;
+        const int64_t slot = pref_slot(tile[r / kPageRows], r % kPageRows);
         if (slot < own.slots) g = own.group[slot];
       }
       rg[r] = g;
@@ -350,11 +380,47 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       w[0] = h;
       w[1] = npg;
       w[2] = static_cast<int32_t>(wl.pages.size());
-      for (int32_t p : touched) {
+      // Column entries in slot order.  Up to four consecutive pages whose
+      // attended rows (over all segments) lie in one 4-row group k, at least
+      // two of them in the list, become one strided entry: the four groups
+      // then cost one 16-column page instead of one page each.
+      auto fold = [](uint64_t m) {
+        return static_cast<uint32_t>((m | (m >> 16) | (m >> 32) | (m >> 48)) & 0xFFFFu);
+      };
+      size_t i = 0;
+      while (i < touched.size()) {
+        const int32_t p = touched[i];
+        const int k = strided ? sub_group(fold(acc[p])) : -1;
+        if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= col.slots) {
+          size_t j = i;
+          bool same = true;
+          while (j < touched.size() && touched[j] <= p + 3) {
+            if (sub_group(fold(acc[touched[j]])) != k) {
+              same = false;
+              break;
+            }
+            ++j;
+          }
+          if (same && j - i >= 2) {
+            uint64_t m = 0;
+            for (size_t x = i; x < j; ++x) {
+              const int jj = touched[x] - p;
+              for (int sg = 0; sg < kMaxSegments; ++sg)
+                m |= ((acc[touched[x]] >> (16 * sg + 4 * k)) & 0xFull) << (16 * sg + 4 * jj);
+              acc[touched[x]] = 0;
+            }
+            wl.pages.push_back(~static_cast<int32_t>(16 * p + 4 * k));
+            wl.masks.push_back(m);
+            i = j;
+            continue;
+          }
+        }
         wl.pages.push_back(p);
         wl.masks.push_back(acc[p]);
         acc[p] = 0;
+        ++i;
       }
+      const size_t n_entries = wl.pages.size() - static_cast<size_t>(w[2]);
       w[3] = static_cast<int32_t>(wl.pages.size());
       for (int i = 0; i < npg; ++i) w[4 + i] = tile[i];
       for (int r = 0; r < kTilePages * kPageRows; ++r) {
@@ -367,7 +433,7 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
         }
         reinterpret_cast<uint32_t*>(w)[12 + r / 8] |= code << (4 * (r % 8));
       }
-      wl.physical_pairs += static_cast<int64_t>(kTilePages * kPageRows) * kPageRows * static_cast<int64_t>(touched.size());
+      wl.physical_pairs += static_cast<int64_t>(kTilePages * kPageRows) * kPageRows * static_cast<int64_t>(n_entries);
       wl.work.insert(wl.work.end(), w, w + kWorkWords);
     }
   }
@@ -489,6 +555,26 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   return SPATTN_OK;
 }
 
+// Rows of one side that no work item writes, as (page, row mask) pairs:
+// pages without a valid slot (all 16 rows), and the rows outside the 4-row
+// group of the pages that a strided owned page stands for (padded rows).
+void fill_list(const Side& s, std::vector<int32_t>& out) {
+  out.clear();
+  std::vector<uint16_t> fill(s.n_pages, 0);
+  for (int64_t p = 0; p < s.n_pages; ++p)
+    if (!s.page_mask[p]) fill[p] = 0xFFFFu;
+  for (const auto& b : owned_blocks(s)) {
+    if (b.strided_group < 0) continue;
+    const int64_t p0 = (~b.pages[0]) / 16;
+    for (int j = 0; j < 4; ++j) fill[p0 + j] = static_cast<uint16_t>(0xFFFFu & ~(0xFu << (4 * b.strided_group)));
+  }
+  for (int64_t p = 0; p < s.n_pages; ++p)
+    if (fill[p]) {
+      out.push_back(static_cast<int32_t>(p));
+      out.push_back(fill[p]);
+    }
+}
+
 template <typename T>
 int upload(const std::vector<T>& host, T** dev, int64_t& bytes) {
   const size_t n = std::max<size_t>(host.size(), 1) * sizeof(T);
@@ -566,8 +652,8 @@ void free_plan_device(spattn_plan_s* P) {
   cudaFree(P->wk.d_work);
   cudaFree(P->wk.d_pages);
   cudaFree(P->wk.d_masks);
-  cudaFree(P->d_q_invalid);
-  cudaFree(P->d_k_invalid);
+  cudaFree(P->d_q_fill);
+  cudaFree(P->d_k_fill);
   cudaFree(P->d_err);
   cudaFree(P->d_delta);
   for (auto& e : P->events) {
@@ -624,10 +710,8 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   st = build_worklist(P->k, P->q, P->bwd_adj, L->heads, L->batch, P->wk);
   if (st) return st;
 
-  for (int64_t p = 0; p < P->q.n_pages; ++p)
-    if (!P->q.page_mask[p]) P->q_invalid_pages.push_back(static_cast<int32_t>(p));
-  for (int64_t p = 0; p < P->k.n_pages; ++p)
-    if (!P->k.page_mask[p]) P->k_invalid_pages.push_back(static_cast<int32_t>(p));
+  fill_list(P->q, P->q_fill);
+  fill_list(P->k, P->k_fill);
 
   P->plan_ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
   if (P->device < 0) return SPATTN_OK;
@@ -639,8 +723,8 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if ((st = upload(P->wk.work, &P->wk.d_work, bytes))) return st;
   if ((st = upload(P->wk.pages, &P->wk.d_pages, bytes))) return st;
   if ((st = upload(P->wk.masks, &P->wk.d_masks, bytes))) return st;
-  if ((st = upload(P->q_invalid_pages, &P->d_q_invalid, bytes))) return st;
-  if ((st = upload(P->k_invalid_pages, &P->d_k_invalid, bytes))) return st;
+  if ((st = upload(P->q_fill, &P->d_q_fill, bytes))) return st;
+  if ((st = upload(P->k_fill, &P->d_k_fill, bytes))) return st;
   if (cudaMalloc(reinterpret_cast<void**>(&P->d_err), sizeof(int)) != cudaSuccess) return SPATTN_ERR_OOM;
   if (cudaMemset(P->d_err, 0, sizeof(int)) != cudaSuccess) return SPATTN_ERR_CUDA;
   const size_t delta_bytes = static_cast<size_t>(L->batch) * L->heads * L->q_slots * sizeof(float);

@@ -18,6 +18,18 @@ constexpr int kTilePages = 8;     // pages per 128-row tile
 constexpr int kMaxSegments = 4;   // distinct groups per work item (16-bit mask each)
 constexpr int kWorkWords = 32;    // int32 words per work item
 
+// Page references (owned pages of a work item, column entries of its list):
+// a value p >= 0 is the 16-row page of slots 16p .. 16p+15; a negative value
+// is a strided page with base slot b = ~value (a multiple of 4), the four
+// 4-row groups b + 16j .. b + 16j + 3 (j = 0..3), row r of it at
+// b + 16 (r / 4) + r % 4.  A strided page gathers rows that sit in the same
+// 4-row group of four consecutive pages, e.g. the single valid dh row of
+// each dt slice of a tile cut by the grid's H edge.
+inline int64_t pref_slot(int32_t ref, int r) {
+  return ref >= 0 ? static_cast<int64_t>(ref) * 16 + r : static_cast<int64_t>(~ref) + 16 * (r >> 2) + (r & 3);
+}
+inline int64_t pref_first_slot(int32_t ref) { return ref >= 0 ? static_cast<int64_t>(ref) * 16 : ~ref; }
+
 // Row codes in a work item (4 bits per tile row).
 constexpr uint32_t kCodeNoSegment = 14;  // owned row without a group (padded): writes zeros
 constexpr uint32_t kCodeNotOwned = 15;   // row written by another item (or beyond the tensor)
@@ -66,10 +78,13 @@ struct spattn_plan_s {
   spattn::Adjacency bwd_adj;  // key group -> query groups
   spattn::WorkList wq;        // query-owned tiles (forward, dQ)
   spattn::WorkList wk;        // key-owned tiles (dK/dV)
-  // pages with no valid row, per side (filled with zeros / -inf)
-  std::vector<int32_t> q_invalid_pages, k_invalid_pages;
-  int32_t* d_q_invalid = nullptr;
-  int32_t* d_k_invalid = nullptr;
+  // Rows that no work item writes, per side, as (page, 16-bit row mask)
+  // pairs: every row of a page with no valid slot, and the padded rows that a
+  // strided owned page leaves out.  The fill kernel writes zeros (and
+  // LSE = -inf) there.
+  std::vector<int32_t> q_fill, k_fill;
+  int32_t* d_q_fill = nullptr;
+  int32_t* d_k_fill = nullptr;
   int* d_err = nullptr;        // device error word
   float* d_delta = nullptr;    // [batch, heads, q_slots] rowsum(dO * O)
   int64_t useful_pairs = 0;

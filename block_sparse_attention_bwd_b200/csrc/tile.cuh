@@ -18,6 +18,13 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
 }
 
+// Slot of row r (0..15) of a page reference: p >= 0 is the page of slots
+// 16p .. 16p+15; a negative value is a strided page with base slot b = ~ref,
+// the four 4-row groups b + 16j .. b + 16j + 3.
+__device__ __forceinline__ int64_t pref_slot(int32_t ref, int r) {
+  return ref >= 0 ? static_cast<int64_t>(ref) * 16 + r : static_cast<int64_t>(~ref) + 16 * (r >> 2) + (r & 3);
+}
+
 // Work item words (see spattn_plan_work in include/spattn.h).
 struct Work {
   int bh, n_own, e0, e1;
@@ -71,14 +78,24 @@ struct StepMasks {
 // request for all chunks.  Each TMA request costs the
 // issuing thread time whatever its size, so fewer, larger boxes keep the
 // producer off the critical path.  All 32 lanes must call this.
+//
+// A strided page (negative reference) is never part of a run: its lane
+// fetches it with one strided 16-row box per 64-column chunk.
 template <int NCH>
 __device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, const TmaPages& maps, int pid, int n,
                                                int bh, uint64_t* bar) {
   const int lane = lane_id();
   const int nxt = __shfl_down_sync(0xffffffffu, pid, 1);
-  const unsigned cont = __ballot_sync(0xffffffffu, lane + 1 < n && nxt == pid + 1);  // bit j: page j+1 follows j
+  // bit j: page j+1 follows page j (both regular)
+  const unsigned cont = __ballot_sync(0xffffffffu, lane + 1 < n && pid >= 0 && nxt == pid + 1);
   const bool start = lane < n && (lane == 0 || !((cont >> (lane - 1)) & 1u));
   if (!start) return;
+  if (pid < 0) {
+    const int base = ~pid;
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) tma_load_5d(dst + c * chunk_bytes + lane * 2048, &maps.m4s, c * 64, 0, 0, base, bh, bar);
+    return;
+  }
   int rem = __ffs(~(cont >> lane));  // run length
   int j = lane;
   if (lane == 0 && rem >= 8 && chunk_bytes == 128 * 128) {

@@ -10,7 +10,7 @@ import block_sparse_attention_bwd_b200 as sp
 import oracle
 from workloads import configs as W
 
-TINY = ["tiny", "tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey"]
+TINY = ["tiny", "tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_hedge"]
 
 
 def _allowed(p, h):
@@ -45,6 +45,17 @@ def test_pair_counts_tiny(name):
         assert st["physical_pairs_dkdv"] >= st["useful_pairs"]
 
 
+def pref_slots(ref):
+    """The 16 slots of a page reference: a page p >= 0 covers 16p .. 16p+15;
+    a negative value is a strided page with base slot b = ~ref, rows
+    b + 16j + r for j, r in 0..3."""
+    ref = int(ref)
+    if ref >= 0:
+        return np.arange(16, dtype=np.int64) + 16 * ref
+    b = ~ref
+    return np.array([b + 16 * (r // 4) + r % 4 for r in range(16)], dtype=np.int64)
+
+
 def _codes(w):
     words = w[12:28].astype(np.int64) & 0xFFFFFFFF
     return np.array([(words[r // 8] >> (4 * (r % 8))) & 0xF for r in range(128)])
@@ -70,13 +81,15 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
         codes = _codes(w)
         pg = pages[e0:e1].astype(np.int64)
         mk = masks[e0:e1].astype(np.uint64)
-        assert np.all(np.diff(pg) > 0), "column pages must be ascending and unique"
+        first = np.array([pref_slots(x)[0] for x in pg], dtype=np.int64)
+        assert np.all(np.diff(first) > 0), "column entries must be in ascending slot order"
+        col_slot = np.stack([pref_slots(x) for x in pg]) if pg.size else np.zeros((0, 16), np.int64)
         for r in range(128):
             c = int(codes[r])
             if c == 15:
                 continue
             assert r < 16 * n_own
-            slot = int(w[4 + r // 16]) * 16 + r % 16
+            slot = int(pref_slots(w[4 + r // 16])[r % 16])
             assert slot < own_group.size
             if row_filter is not None and slot not in row_filter:
                 continue
@@ -86,7 +99,7 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
                 continue
             assert c < 4 and own_group[slot] >= 0
             bits = ((mk[:, None] >> (np.uint64(16 * c) + bits16)) & np.uint64(1)).astype(bool)
-            cols = (pg[:, None] * 16 + np.arange(16))[bits]
+            cols = col_slot[bits]
             assert np.all(cols < col_slots)
             for col in cols.tolist():
                 pairs[(h, slot, col)] = pairs.get((h, slot, col), 0) + 1
@@ -112,8 +125,13 @@ def test_coverage_invariant_tiny(name, which):
                 got[i, j] = True
         assert np.array_equal(got, M)
         for slot in range(own_group.size):
-            expect = 1 if valid_pages[slot // 16] else 0
-            assert owned.get((h, slot), 0) == expect, (h, slot)
+            # every valid slot is owned exactly once; a padded slot at most once
+            # (the padded rows a strided owned page leaves out are filled instead)
+            n = owned.get((h, slot), 0)
+            if own_group[slot] >= 0:
+                assert n == 1, (h, slot)
+            else:
+                assert n <= (1 if valid_pages[slot // 16] else 0), (h, slot)
 
 
 @pytest.mark.parametrize("name", ["full", "partial", "vsa", "svg2"])
@@ -166,3 +184,40 @@ def test_plan_independent_of_thread_count(name, monkeypatch):
     sa, sb = plans[0].stats(), plans[1].stats()
     for k in ("useful_pairs", "physical_pairs_fwd", "physical_pairs_dkdv", "n_work_fwd", "n_entries_dkdv"):
         assert sa[k] == sb[k], k
+
+
+def test_strided_pages_are_formed_where_rows_share_a_group():
+    """tiny_hedge's H-edge tiles: four pages with valid rows 0..3 each become
+    one strided owned page, and their key pages one strided column entry."""
+    p = W.make_problem("tiny_hedge")
+    pl = sp.Plan.from_problem(p)
+    for which in (0, 1):
+        work, pages, _ = pl.work(which)
+        assert (pages < 0).any(), which
+        owned = work[:, 4:12][np.arange(8)[None, :] < work[:, 1:2]]
+        assert (owned < 0).any(), which
+        for ref in np.concatenate([pages[pages < 0], owned[owned < 0]]):
+            slots = pref_slots(ref)
+            assert (p.kv_group[slots] >= 0).all() if which == 0 and ref in pages else True
+            assert slots.max() < p.q_slots
+
+
+def test_strided_pages_stay_inside_the_tensor():
+    """Key rows 12..15 of every page valid, 62 slots: a strided page over the
+    4-row group 12..15 of pages 0..3 would reach slots 60..63, past the end of
+    the tensor, so none may cover a slot >= 62."""
+    kg = np.full(62, -1, np.int32)
+    for j in range(4):
+        kg[16 * j + 12:16 * j + 16] = 0
+    kg = kg[:62]
+    qg = np.zeros(16, np.int32)
+    pl = sp.Plan(qg, kg, 1, 1, np.array([0, 1], np.int64), np.array([0], np.int32), batch=1, heads=1, head_dim=64)
+    for which in (0, 1):
+        work, pages, _ = pl.work(which)
+        refs = list(pages) + list(work[:, 4:12][np.arange(8)[None, :] < work[:, 1:2]])
+        for ref in refs:
+            assert pref_slots(ref).max() < 62 or int(ref) >= 0, ref
+    # the allowed pairs are still covered exactly once
+    pairs, _ = _covered(W.Problem("ragged", 1, 1, 64, qg, kg, 1, 1, np.array([0, 1], np.int64),
+                                  np.array([0], np.int32), 0), pl, 0)
+    assert sorted(j for (_, _, j) in pairs) == sorted(np.nonzero(kg >= 0)[0].tolist() * 16)

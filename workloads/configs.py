@@ -57,7 +57,7 @@ import numpy as np
 PAD_SENTINEL = 1000.0
 
 CONFIG_NAMES = ("tiny", "full", "partial", "vsa", "svg2")
-EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_nokeys")
+EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_nokeys", "tiny_hedge")
 
 
 @dataclasses.dataclass
@@ -253,6 +253,14 @@ def make_problem(name: str) -> Problem:
         row_ptr, cols = _csr(rows)
         return Problem(name, 1, 2, 64, group, group.copy(), 12, 12, row_ptr, cols, 15000,
                        "tiny STA; head 1 attends nothing (empty column lists)")
+    if name == "tiny_hedge":
+        # 4x5x12 grid: the tiles of the second tile row in H hold a single dh
+        # row, so each of their four pages has 4 valid rows in the same 4-row
+        # group (the case the strided pages compact); clamped 1x2x2 window
+        group, tiles = sta_layout((4, 5, 12))
+        row_ptr, cols = sta_graph(tiles, (1, 2, 2), 2)
+        return Problem(name, 1, 2, 64, group, group.copy(), 6, 6, row_ptr, cols, 16000,
+                       "tiny STA whose H-edge tiles keep one dh row (strided pages)")
     raise KeyError(name)
 
 
