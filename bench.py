@@ -309,6 +309,26 @@ def run_reference(args):
     return 0
 
 
+def device_plan_ms(plan, p, dev, reps=5):
+    """Median wall time of re-planning the workload's graph on the device
+    (spattn_plan_set_graph_device, one stream synchronisation included).
+    It switches the plan to slot-order tiles, so it runs after the timed
+    steps."""
+    import torch
+
+    rp = torch.from_numpy(np.ascontiguousarray(p.row_ptr, dtype=np.int64)).to(dev)
+    cols = torch.from_numpy(np.ascontiguousarray(p.kv_groups, dtype=np.int32)).to(dev)
+    plan.set_graph_device(rp, cols)  # first call allocates the planner's device state
+    times = []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        plan.set_graph_device(rp, cols)
+        torch.cuda.synchronize()
+        times.append((time.perf_counter() - t0) * 1e3)
+    return statistics.median(times)
+
+
 def measure_workload(name, steps, warmup, dev, peak_burst):
     """fwd and fwd+bwd useful-pair TFLOP/s of one workload on resident inputs
     (CUDA events on the launch stream, L2 flushed between steps when the
@@ -367,6 +387,7 @@ def measure_workload(name, steps, warmup, dev, peak_burst):
            "useful_over_physical_dkdv": U / st["physical_pairs_dkdv"], "useful_over_bsa_64x64": U / st["bsa_pairs"],
            "plan_ms": st["plan_ms"], "sm_mhz": clk["sm_mhz"], "clock_reasons": clk["reasons"],
            "l2": "flushed between steps" if flush else "inputs larger than L2"}
+    res["device_plan_ms"] = device_plan_ms(plan, p, dev)
     plan.close()
     del x, out, scratch
     torch.cuda.empty_cache()
@@ -549,6 +570,8 @@ def run_ours(args):
                           f"extrapolated linearly by useful pairs to the whole workload"),
                "fwd_value": 4 * D * U / tf / 1e12}
 
+    dplan_ms = device_plan_ms(plan, p, dev) if rank == 0 else None
+
     # ---------------- every other large workload, measured the same way ----------------
     workloads = None
     if rank == 0 and world == 1 and args.other_workloads:
@@ -578,6 +601,7 @@ def run_ours(args):
                   "useful_over_physical_fwd": U / st["physical_pairs_fwd"]},
         "kernels": kern,
         "plan_ms": st["plan_ms"],
+        "device_plan_ms": dplan_ms,
         "roofline": roofline,
         "cpu_baseline": cpu,
         "e2e": e2e,

@@ -38,7 +38,7 @@ STATUS_NAMES = {
 ENTRY_POINTS = (
     "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_bwd_noalloc", "spattn_check", "spattn_plan_stats", "spattn_profile",
     "spattn_profile_read", "spattn_plan_pages", "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy",
-    "spattn_status_string", "spattn_wait_selftest",
+    "spattn_status_string", "spattn_wait_selftest", "spattn_plan_set_graph_device", "spattn_plan_entry_heads",
 )
 
 
@@ -54,6 +54,7 @@ class _Layout(ctypes.Structure):
         ("q_slots", ctypes.c_int64), ("kv_slots", ctypes.c_int64),
         ("q_group", ctypes.POINTER(ctypes.c_int32)), ("kv_group", ctypes.POINTER(ctypes.c_int32)),
         ("n_q_groups", ctypes.c_int32), ("n_kv_groups", ctypes.c_int32), ("scale", ctypes.c_float),
+        ("kv_heads", ctypes.c_int32), ("graph_batches", ctypes.c_int32),
     ]
 
 
@@ -92,12 +93,15 @@ def _lib():
         lib.spattn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
         lib.spattn_check.argtypes = [P, P]
         lib.spattn_wait_selftest.argtypes = [P, I64, P]
+        lib.spattn_plan_set_graph_device.argtypes = [P, P, P, I64, P]
         lib.spattn_plan_stats.argtypes = [P, ctypes.POINTER(_Stats)]
         lib.spattn_plan_pages.argtypes = [P, I32, I64, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64)]
         lib.spattn_plan_qblocks.argtypes = [P, I32, I64, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64)]
         lib.spattn_plan_work.argtypes = [P, I32, ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(I64),
                                          ctypes.POINTER(ctypes.POINTER(I32)), ctypes.POINTER(ctypes.POINTER(ctypes.c_uint64)),
                                          ctypes.POINTER(I64)]
+        lib.spattn_plan_entry_heads.argtypes = [P, I32, ctypes.POINTER(ctypes.POINTER(ctypes.c_uint16)),
+                                                ctypes.POINTER(I64)]
         lib.spattn_profile.argtypes = [P, ctypes.c_int]
         lib.spattn_profile_read.argtypes = [P, ctypes.POINTER(_KernelTimes)]
         lib.spattn_plan_destroy.argtypes = [P]
@@ -129,27 +133,32 @@ class Plan:
     """
 
     def __init__(self, q_group, kv_group, n_q_groups, n_kv_groups, row_ptr, kv_groups, *, batch, heads,
-                 head_dim, scale=0.0):
+                 head_dim, scale=0.0, kv_heads=0, graph_batches=1):
         qg, kg = _i32(q_group), _i32(kv_group)
         rp = np.ascontiguousarray(row_ptr, dtype=np.int64)
         cols = _i32(kv_groups) if len(kv_groups) else np.zeros(1, np.int32)
         self._keep = (qg, kg, rp, cols)
         lay = _Layout(batch, heads, head_dim, qg.size, kg.size,
                       qg.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), kg.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)),
-                      int(n_q_groups), int(n_kv_groups), float(scale))
+                      int(n_q_groups), int(n_kv_groups), float(scale), int(kv_heads), int(graph_batches))
         gr = _Graph(rp.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), cols.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
         h = ctypes.c_void_p()
         _check(_lib().spattn_plan(ctypes.byref(lay), ctypes.byref(gr), ctypes.byref(h)), "spattn_plan")
         self.handle = h
         self.batch, self.heads, self.head_dim = batch, heads, head_dim
+        self.kv_heads = heads if kv_heads == 0 else kv_heads
         self.q_slots, self.kv_slots = qg.size, kg.size
         self._keep = None
 
     @classmethod
     def from_problem(cls, problem, batch: Optional[int] = None):
+        b = problem.batch if batch is None else batch
+        gb = getattr(problem, "graph_batches", 1)
+        if gb != 1 and b != problem.batch:
+            raise ValueError("a problem with one graph per batch entry has a fixed batch")
         return cls(problem.q_group, problem.kv_group, problem.n_q_groups, problem.n_kv_groups, problem.row_ptr,
-                   problem.kv_groups, batch=problem.batch if batch is None else batch, heads=problem.heads,
-                   head_dim=problem.head_dim, scale=problem.scale)
+                   problem.kv_groups, batch=b, heads=problem.heads, head_dim=problem.head_dim, scale=problem.scale,
+                   kv_heads=getattr(problem, "kv_heads", 0) or 0, graph_batches=gb)
 
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:
@@ -161,6 +170,19 @@ class Plan:
             self.close()
         except Exception:
             pass
+
+    def set_graph_device(self, row_ptr, kv_groups, stream=None):
+        """Re-plan on the GPU for a new graph: ``row_ptr`` int64 and
+        ``kv_groups`` int32, contiguous CUDA tensors in the spattn_graph
+        format (spattn_plan_set_graph_device)."""
+        import torch
+
+        if row_ptr.dtype != torch.int64 or not row_ptr.is_cuda or not row_ptr.is_contiguous():
+            raise ValueError("row_ptr: expected a contiguous CUDA int64 tensor")
+        if kv_groups.dtype != torch.int32 or not kv_groups.is_cuda or not kv_groups.is_contiguous():
+            raise ValueError("kv_groups: expected a contiguous CUDA int32 tensor")
+        _check(_lib().spattn_plan_set_graph_device(self.handle, _ptr(row_ptr), _ptr(kv_groups), kv_groups.numel(),
+                                                   _stream_handle(stream)), "spattn_plan_set_graph_device")
 
     def stats(self) -> dict:
         s = _Stats()
@@ -189,6 +211,10 @@ class Plan:
         _check(_lib().spattn_plan_qblocks(self.handle, head, page, ctypes.byref(ptr), ctypes.byref(n)), "spattn_plan_qblocks")
         return np.ctypeslib.as_array(ptr, shape=(n.value,)).copy() if n.value else np.zeros(0, np.int32)
 
+    def entry_heads(self, which: int) -> np.ndarray:
+        """Per entry of work list ``which``: its query head relative to the item's K/V head group."""
+        return _entry_heads(self, which)
+
     def work(self, which: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
         """(work [n, 32] int32, pages [e] int32, masks [e] uint64) of pass ``which`` (0 query-owned, 1 key-owned)."""
         w = ctypes.POINTER(ctypes.c_int32)()
@@ -201,6 +227,14 @@ class Plan:
         pages = np.ctypeslib.as_array(p, shape=(ne.value,)).copy() if ne.value else np.zeros(0, np.int32)
         masks = np.ctypeslib.as_array(m, shape=(ne.value,)).copy() if ne.value else np.zeros(0, np.uint64)
         return work, pages, masks
+
+
+def _entry_heads(plan, which):
+    h = ctypes.POINTER(ctypes.c_uint16)()
+    n = ctypes.c_int64()
+    _check(_lib().spattn_plan_entry_heads(plan.handle, which, ctypes.byref(h), ctypes.byref(n)),
+           "spattn_plan_entry_heads")
+    return np.ctypeslib.as_array(h, shape=(n.value,)).copy() if n.value else np.zeros(0, np.uint16)
 
 
 def _stream_handle(stream):
@@ -227,7 +261,7 @@ def spattn_fwd(q, k, v, plan: Plan, o=None, lse=None, stream=None):
     import torch
 
     qs = (plan.batch, plan.heads, plan.q_slots, plan.head_dim)
-    ks = (plan.batch, plan.heads, plan.kv_slots, plan.head_dim)
+    ks = (plan.batch, plan.kv_heads, plan.kv_slots, plan.head_dim)
     _need(q, "q", qs, torch.bfloat16)
     _need(k, "k", ks, torch.bfloat16)
     _need(v, "v", ks, torch.bfloat16)
@@ -247,7 +281,7 @@ def spattn_bwd(q, k, v, o, lse, do, plan: Plan, dq=None, dk=None, dv=None, strea
     import torch
 
     qs = (plan.batch, plan.heads, plan.q_slots, plan.head_dim)
-    ks = (plan.batch, plan.heads, plan.kv_slots, plan.head_dim)
+    ks = (plan.batch, plan.kv_heads, plan.kv_slots, plan.head_dim)
     for t, nm, sh in ((q, "q", qs), (k, "k", ks), (v, "v", ks), (o, "o", qs), (do, "do", qs)):
         _need(t, nm, sh, torch.bfloat16)
     _need(lse, "lse", qs[:3], torch.float32)

@@ -17,6 +17,8 @@ void free_plan_device(spattn_plan_s* P);
 void canonical_pages(const spattn_plan_s& P, int32_t h, int64_t qb, std::vector<int32_t>& out);
 void transposed_qblocks(const spattn_plan_s& P, int32_t h, int64_t page, std::vector<int32_t>& out);
 int64_t bsa_pairs(const spattn_plan_s& P);
+int refresh_host(spattn_plan_s* P);
+int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_groups, int64_t nnz, cudaStream_t st);
 
 namespace {
 
@@ -136,6 +138,10 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
   a.col_slots = col_slots;
   a.scale = P->scale;
   a.err = P->d_err;
+  a.heads = P->heads;
+  a.kv_heads = P->kv_heads;
+  a.kv_group = P->heads / P->kv_heads;
+  a.col_heads = w.d_heads;
   return a;
 }
 
@@ -192,9 +198,10 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return SPATTN_ERR_INVALID_ARG;
   const int D = plan->head_dim;
   const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
+  const int64_t bh_kv = static_cast<int64_t>(plan->batch) * plan->kv_heads;
   TmaPages tq, tk, tv;
-  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh) ||
-      !make_pages(&tv, v, D, plan->k.slots, bh))
+  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh_kv) ||
+      !make_pages(&tv, v, D, plan->k.slots, bh_kv))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* O = static_cast<__nv_bfloat16*>(o);
@@ -219,9 +226,10 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
     return SPATTN_ERR_INVALID_ARG;
   const int D = plan->head_dim;
   const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
+  const int64_t bh_kv = static_cast<int64_t>(plan->batch) * plan->kv_heads;
   TmaPages tq, tk, tv, tdo;
-  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh) ||
-      !make_pages(&tv, v, D, plan->k.slots, bh) || !make_pages(&tdo, d_o, D, plan->q.slots, bh))
+  if (!make_pages(&tq, q, D, plan->q.slots, bh) || !make_pages(&tk, k, D, plan->k.slots, bh_kv) ||
+      !make_pages(&tv, v, D, plan->k.slots, bh_kv) || !make_pages(&tdo, d_o, D, plan->q.slots, bh))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* dQ = static_cast<__nv_bfloat16*>(dq);
@@ -243,7 +251,7 @@ int spattn_bwd(const void* q, const void* k, const void* v, const void* o, const
     });
   if (e == cudaSuccess && !plan->k_fill.empty())
     e = timed(plan, SPATTN_K_FILL, s, [&] {
-      return launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh, plan->k.slots, dK,
+      return launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh_kv, plan->k.slots, dK,
                          dV, nullptr, s);
     });
   if (e == cudaSuccess && !plan->q_fill.empty())
@@ -275,14 +283,31 @@ int spattn_check(spattn_plan_t plan, void* stream) {
   return h == 1 ? SPATTN_ERR_TIMEOUT : SPATTN_ERR_DEVICE;
 }
 
+int spattn_plan_set_graph_device(spattn_plan_t plan, const int64_t* row_ptr, const int32_t* kv_groups, int64_t nnz,
+                                 void* stream) {
+  if (!plan || !row_ptr || nnz < 0 || (nnz > 0 && !kv_groups)) return SPATTN_ERR_INVALID_ARG;
+  const int st = check_plan_device(plan);
+  if (st) return st;
+  if (plan->kv_heads != plan->heads || plan->graph_batches != 1) return SPATTN_ERR_UNSUPPORTED;
+  try {
+    return device_replan(plan, row_ptr, kv_groups, nnz, static_cast<cudaStream_t>(stream));
+  } catch (...) {
+    return SPATTN_ERR_OOM;
+  }
+}
+
 int spattn_plan_stats(spattn_plan_t plan, spattn_stats* s) {
   if (!plan || !s) return SPATTN_ERR_INVALID_ARG;
+  {
+    const int st = refresh_host(plan);
+    if (st) return st;
+  }
   if (plan->bsa_pairs < 0) plan->bsa_pairs = bsa_pairs(*plan);
   std::memset(s, 0, sizeof(*s));
   s->useful_pairs = plan->useful_pairs;
-  s->physical_pairs_fwd = plan->wq.physical_pairs * plan->batch;
-  s->physical_pairs_dq = plan->wq.physical_pairs * plan->batch;
-  s->physical_pairs_dkdv = plan->wk.physical_pairs * plan->batch;
+  s->physical_pairs_fwd = plan->wq.physical_pairs;
+  s->physical_pairs_dq = plan->wq.physical_pairs;
+  s->physical_pairs_dkdv = plan->wk.physical_pairs;
   s->bsa_pairs = plan->bsa_pairs;
   s->n_work_fwd = plan->wq.n_work;
   s->n_work_dkdv = plan->wk.n_work;
@@ -322,7 +347,11 @@ int spattn_profile_read(spattn_plan_t plan, spattn_kernel_times* out) {
 }
 
 int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const int32_t** pages, int64_t* n) {
-  if (!plan || !pages || !n || head < 0 || head >= plan->heads || qblock < 0 ||
+  if (plan) {
+    const int st = refresh_host(plan);
+    if (st) return st;
+  }
+  if (!plan || !pages || !n || head < 0 || head >= plan->graph_batches * plan->heads || qblock < 0 ||
       qblock >= (plan->q.slots + kBlockRows - 1) / kBlockRows)
     return SPATTN_ERR_INVALID_ARG;
   canonical_pages(*plan, head, qblock, plan->scratch);
@@ -332,7 +361,12 @@ int spattn_plan_pages(spattn_plan_t plan, int32_t head, int64_t qblock, const in
 }
 
 int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const int32_t** qblocks, int64_t* n) {
-  if (!plan || !qblocks || !n || head < 0 || head >= plan->heads || page < 0 || page >= plan->k.n_pages)
+  if (plan) {
+    const int st = refresh_host(plan);
+    if (st) return st;
+  }
+  if (!plan || !qblocks || !n || head < 0 || head >= plan->graph_batches * plan->heads || page < 0 ||
+      page >= plan->k.n_pages)
     return SPATTN_ERR_INVALID_ARG;
   transposed_qblocks(*plan, head, page, plan->scratch);
   *qblocks = plan->scratch.data();
@@ -342,6 +376,10 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
 
 int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work, const int32_t** pages,
                      const uint64_t** masks, int64_t* n_entries) {
+  if (plan) {
+    const int st = refresh_host(plan);
+    if (st) return st;
+  }
   if (!plan || !work || !n_work || !pages || !masks || !n_entries || (which != 0 && which != 1))
     return SPATTN_ERR_INVALID_ARG;
   const WorkList& w = which == 0 ? plan->wq : plan->wk;
@@ -350,6 +388,17 @@ int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, in
   *pages = w.pages.data();
   *masks = w.masks.data();
   *n_entries = static_cast<int64_t>(w.pages.size());
+  return SPATTN_OK;
+}
+
+int spattn_plan_entry_heads(spattn_plan_t plan, int32_t which, const uint16_t** heads, int64_t* n_entries) {
+  if (!plan || !heads || !n_entries || (which != 0 && which != 1)) return SPATTN_ERR_INVALID_ARG;
+  const int st = refresh_host(plan);
+  if (st) return st;
+  WorkList& w = which == 0 ? plan->wq : plan->wk;
+  if (w.heads.size() != w.pages.size()) w.heads.assign(w.pages.size(), 0);  // lists rebuilt on the device
+  *heads = w.heads.data();
+  *n_entries = static_cast<int64_t>(w.heads.size());
   return SPATTN_OK;
 }
 

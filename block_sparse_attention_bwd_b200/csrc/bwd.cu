@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                 const uint64_t* __restrict__ col_masks, const float* __restrict__ lse,
                 const float* __restrict__ delta, __nv_bfloat16* __restrict__ out_dk,
                 __nv_bfloat16* __restrict__ out_dv, int64_t kv_slots, int64_t q_slots, float sl2, float scale,
-                int* err) {
+                int heads, int kv_heads, int kv_group, const uint16_t* __restrict__ col_heads, int* err) {
   using C = DkvCfg<D>;
   constexpr int QS = C::kQStages, DS = C::kDStages, NP = kBwdStepPages, SP = C::kStagePages;
   constexpr int SPS = SP / NP;       // steps per stage
@@ -255,19 +255,29 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     auto page_id = [&](int t) {
       return (t < n_stages && lane < min(SP, n_cols - t * SP)) ? __ldg(col_pages + wk.e0 + t * SP + lane) : 0;
     };
+    // Query head of a column page: the item's K/V head owns the query heads
+    // q_base .. q_base + kv_group - 1 (grouped-query attention); each entry
+    // names its offset.
+    const int q_base = (wk.bh / kv_heads) * heads + (wk.bh % kv_heads) * kv_group;
+    auto col_bh = [&](int t) {
+      return q_base + ((col_heads && t < n_stages && lane < min(SP, n_cols - t * SP))
+                           ? static_cast<int>(__ldg(col_heads + wk.e0 + t * SP + lane))
+                           : 0);
+    };
     // Raw loads only (nothing here reads the loaded registers); a dead column
     // (beyond the step or the tensor) loads a valid address and is zeroed
     // where the value is used, through its bit in `live`.
-    auto fetch_terms = [&](int t, int pg_lane, float (&x)[NH], uint32_t& live) {
+    auto fetch_terms = [&](int t, int pg_lane, int bh_lane, float (&x)[NH], uint32_t& live) {
       const int n_t = min(SP, n_cols - t * SP);
       live = 0u;
 #pragma unroll
       for (int h = 0; h < NH; ++h) {
         const int idx = lane + 32 * h;  // column of the stage
         const int pg = __shfl_sync(0xffffffffu, pg_lane, idx >> 4);
+        const int cb = __shfl_sync(0xffffffffu, bh_lane, idx >> 4);
         const int64_t slot = pref_slot(pg, idx & 15);
         const bool ok = t < n_stages && (idx >> 4) < n_t && slot < q_slots;
-        x[h] = __ldg(terms + static_cast<int64_t>(wk.bh) * q_slots + (ok ? slot : 0));
+        x[h] = __ldg(terms + static_cast<int64_t>(cb) * q_slots + (ok ? slot : 0));
         live |= ok ? (1u << h) : 0u;
       }
     };
@@ -279,17 +289,19 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       return aug_row(ok && isfinite(x) ? x : 0.f);
     };
     int pid = page_id(0), pid_next = page_id(1);
+    int cbh = col_bh(0), cbh_next = col_bh(1);
     float xc[NH];
     uint32_t livec;
-    fetch_terms(0, pid, xc, livec);
+    fetch_terms(0, pid, cbh, xc, livec);
     int issued = 0;
     for (int t = 0; t < n_stages; ++t) {
       const int s = t % NS;
       const int n = min(SP, n_cols - t * SP);
       const int pid_next2 = page_id(t + 2);
+      const int cbh_next2 = col_bh(t + 2);
       float xn[NH];
       uint32_t liven;
-      fetch_terms(t + 1, pid_next, xn, liven);
+      fetch_terms(t + 1, pid_next, cbh_next, xn, liven);
       if (t >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((t / NS) - 1) & 1, ab))) break;
 #pragma unroll
       for (int h = 0; h < NH; ++h)
@@ -298,10 +310,12 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
+      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, cbh, &full[s]);
       issued = t + 1;
       pid = pid_next;
       pid_next = pid_next2;
+      cbh = cbh_next;
+      cbh_next = cbh_next2;
       livec = liven;
 #pragma unroll
       for (int h = 0; h < NH; ++h) xc[h] = xn[h];
@@ -520,7 +534,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
               const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
               const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
               const uint64_t* __restrict__ col_masks, const float* __restrict__ lse, const float* __restrict__ delta,
-              __nv_bfloat16* __restrict__ out_dq, int64_t q_slots, float sl2, float scale, int* err) {
+              __nv_bfloat16* __restrict__ out_dq, int64_t q_slots, float sl2, float scale, int heads, int kv_group,
+              int* err) {
   using C = DqCfg<D>;
   constexpr int KS = C::kKStages, VS = C::kVStages, NP = kBwdStepPages, SP = C::kStagePages;
   constexpr int SPS = SP / NP;  // steps per stage
@@ -548,6 +563,8 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   const Abort ab{abort_flag, err};
 
   const Work wk = load_work(work, blockIdx.x);
+  // K/V head of this item's query head (grouped-query attention)
+  const int kv_bh = (wk.bh / heads) * (heads / kv_group) + (wk.bh % heads) / kv_group;
   const int n_cols = wk.e1 - wk.e0;
   const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
@@ -621,7 +638,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
       if (t >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((t / NS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, wk.bh, &full[s]);
+      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, kv_bh, &full[s]);
       issued = t + 1;
     }
     if (lane == 0) {
@@ -845,7 +862,7 @@ static cudaError_t launch_dkdv_t(const TmaPages& tk, const TmaPages& tv, const T
   if (e != cudaSuccess || a.n_work == 0) return e;
   dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), kDkvThreads, C::kSmem, st>>>(
       tk, tv, tq, tdo, a.work, a.pages, a.masks, lse, delta, dk, dv, a.own_slots, a.col_slots, a.scale * kLog2e,
-      a.scale, a.err);
+      a.scale, a.heads, a.kv_heads, a.kv_group, a.col_heads, a.err);
   return cudaGetLastError();
 }
 
@@ -857,7 +874,8 @@ static cudaError_t launch_dq_t(const __nv_bfloat16* q, const TmaPages& tdo, cons
   cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
   dq_kernel<D><<<static_cast<unsigned>(a.n_work), kDkvThreads, C::kSmem, st>>>(
-      q, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.err);
+      q, tdo, tk, tv, a.work, a.pages, a.masks, lse, delta, dq, a.own_slots, a.scale * kLog2e, a.scale, a.heads,
+      a.kv_group, a.err);
   return cudaGetLastError();
 }
 

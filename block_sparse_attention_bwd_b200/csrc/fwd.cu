@@ -56,7 +56,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
                const __grid_constant__ TmaPages tm_v, const int32_t* __restrict__ work,
                const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
                __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
-               int* err) {
+               int heads, int kv_group, int* err) {
   using C = FwdCfg<D>;
   constexpr int KS = C::kKStages, VS = C::kVStages, NP = kFwdStepPages;
   extern __shared__ uint8_t smem_raw[];
@@ -79,6 +79,8 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   const Abort ab{abort_flag, err};
 
   const Work wk = load_work(work, blockIdx.x);
+  // K/V head of this item's query head (grouped-query attention)
+  const int kv_bh = (wk.bh / heads) * (heads / kv_group) + (wk.bh % heads) / kv_group;
   const int n_cols = wk.e1 - wk.e0;
   const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
@@ -134,12 +136,12 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(sK + ks * C::kStage, kFwdStageChunk, tm_k, pid, n, wk.bh, &k_full[ks]);
+      load_page_runs<C::kNch>(sK + ks * C::kStage, kFwdStageChunk, tm_k, pid, n, kv_bh, &k_full[ks]);
       k_issued = st + 1;
       if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(sV + vs * C::kStage, kFwdStageChunk, tm_v, pid, n, wk.bh, &v_full[vs]);
+      load_page_runs<C::kNch>(sV + vs * C::kStage, kFwdStageChunk, tm_v, pid, n, kv_bh, &v_full[vs]);
       v_issued = st + 1;
     }
     // no copy may still be landing in shared memory when the CTA exits
@@ -365,7 +367,7 @@ cudaError_t launch_fwd_t(const TmaPages& tq, const TmaPages& tk, const TmaPages&
   if (e != cudaSuccess) return e;
   if (a.n_work == 0) return cudaSuccess;
   fwd_kernel<D><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
-      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.err);
+      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.heads, a.kv_group, a.err);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,11 @@ struct TileArgs {
   int64_t col_slots = 0;            // rows per (batch, head) of the column side
   float scale = 0.f;                // softmax scale
   int* err = nullptr;               // device error word
+  // Grouped-query attention: query head h reads K/V head h / kv_group
+  // (heads = query heads, kv_heads = heads / kv_group).  For the key-owned
+  // pass, entry e's column head is the item's first query head + col_heads[e].
+  int heads = 1, kv_heads = 1, kv_group = 1;
+  const uint16_t* col_heads = nullptr;
 };
 
 // K1: O, LSE for every query-owned work item.

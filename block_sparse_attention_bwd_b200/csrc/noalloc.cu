@@ -71,9 +71,10 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
   int st = scratch_address(&delta);
   if (st) return st;
   const int D = plan->head_dim;
+  const int64_t bh_kv = static_cast<int64_t>(plan->batch) * plan->kv_heads;
   TmaPages tq, tk, tv, tdo;
-  if (!make_tensor_pages(&tq, q, D, plan->q.slots, bh) || !make_tensor_pages(&tk, k, D, plan->k.slots, bh) ||
-      !make_tensor_pages(&tv, v, D, plan->k.slots, bh) || !make_tensor_pages(&tdo, d_o, D, plan->q.slots, bh))
+  if (!make_tensor_pages(&tq, q, D, plan->q.slots, bh) || !make_tensor_pages(&tk, k, D, plan->k.slots, bh_kv) ||
+      !make_tensor_pages(&tv, v, D, plan->k.slots, bh_kv) || !make_tensor_pages(&tdo, d_o, D, plan->q.slots, bh))
     return SPATTN_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   auto* dQ = static_cast<__nv_bfloat16*>(dq);
@@ -89,7 +90,7 @@ extern "C" int spattn_bwd_noalloc(const void* q, const void* k, const void* v, c
   if (e == cudaSuccess)
     e = launch_dq(D, static_cast<const __nv_bfloat16*>(q), tdo, tk, tv, make_tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), lse, delta, dQ, s);
   if (e == cudaSuccess && !plan->k_fill.empty())
-    e = launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh, plan->k.slots, dK, dV,
+    e = launch_fill(D, plan->d_k_fill, static_cast<int64_t>(plan->k_fill.size() / 2), bh_kv, plan->k.slots, dK, dV,
                     nullptr, s);
   if (e == cudaSuccess && !plan->q_fill.empty())
     e = launch_fill(D, plan->d_q_fill, static_cast<int64_t>(plan->q_fill.size() / 2), bh, plan->q.slots, dQ,

@@ -31,6 +31,7 @@
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
+#include <functional>
 #include <iterator>
 #include <new>
 #include <queue>
@@ -38,6 +39,11 @@
 #include <tuple>
 
 namespace spattn {
+
+bool strided_setting() {
+  const char* env = std::getenv("SPATTN_PLAN_STRIDED");
+  return !(env && env[0] == '0');
+}
 
 namespace {
 
@@ -133,10 +139,7 @@ int sub_group(uint32_t m) {
 }
 
 // Strided pages are used unless SPATTN_PLAN_STRIDED=0 (for comparisons).
-bool strided_enabled() {
-  const char* env = std::getenv("SPATTN_PLAN_STRIDED");
-  return !(env && env[0] == '0');
-}
+bool strided_enabled() { return strided_setting(); }
 
 // A 64-slot block of the owned side: references to its valid pages (one
 // strided page when all four pages are valid and their valid rows share a
@@ -216,24 +219,33 @@ size_t union_size(const std::vector<int32_t>& a, const std::vector<int32_t>& b) 
 // the pages of each group) merges first, while the merged cluster holds at
 // most 8 pages and at most 4 groups (one work item).  Clusters left with room
 // are then filled in slot order under the same limits.
-std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency& adj, int32_t h,
+std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency& adj,
+                                               const std::vector<int64_t>& src_heads,
                                                const std::vector<OwnBlock>& blocks) {
   const int32_t nb = static_cast<int32_t>(blocks.size());
+  const int32_t ng = col.n_groups;
+  const int64_t n_codes = static_cast<int64_t>(ng) * static_cast<int64_t>(src_heads.size());
+  // a block's signature: (head offset j, column group) pairs as j * ng + group
   std::vector<std::vector<int32_t>> sig(nb);
   for (int32_t b = 0; b < nb; ++b) {
-    for (int32_t g : blocks[b].groups) {
-      const int64_t r = static_cast<int64_t>(h) * adj.n_src + g;
-      sig[b].insert(sig[b].end(), adj.dst.begin() + adj.ptr[r], adj.dst.begin() + adj.ptr[r + 1]);
-    }
+    for (size_t j = 0; j < src_heads.size(); ++j)
+      for (int32_t g : blocks[b].groups) {
+        const int64_t r = src_heads[j] * adj.n_src + g;
+        for (int64_t e = adj.ptr[r]; e < adj.ptr[r + 1]; ++e)
+          sig[b].push_back(static_cast<int32_t>(j * ng + adj.dst[e]));
+      }
     std::sort(sig[b].begin(), sig[b].end());
     sig[b].erase(std::unique(sig[b].begin(), sig[b].end()), sig[b].end());
   }
-  auto wt = [&](int32_t g) { return col.gp_ptr[g + 1] - col.gp_ptr[g]; };
-  // column group -> blocks whose signature holds it
-  std::vector<int64_t> ip(static_cast<size_t>(col.n_groups) + 1, 0);
+  auto wt = [&](int32_t code) {
+    const int32_t g = code % ng;
+    return col.gp_ptr[g + 1] - col.gp_ptr[g];
+  };
+  // signature code -> blocks whose signature holds it
+  std::vector<int64_t> ip(static_cast<size_t>(n_codes) + 1, 0);
   for (int32_t b = 0; b < nb; ++b)
     for (int32_t g : sig[b]) ip[g + 1] += 1;
-  for (int32_t g = 0; g < col.n_groups; ++g) ip[g + 1] += ip[g];
+  for (int64_t g = 0; g < n_codes; ++g) ip[g + 1] += ip[g];
   std::vector<int32_t> iv(ip.back());
   {
     std::vector<int64_t> fill(ip.begin(), ip.end() - 1);
@@ -341,9 +353,14 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
 }
 
 // Work items of one head for one pass; work words use bh = head (batch 0).
-void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t h,
-                const std::vector<std::vector<int32_t>>& tiles, WorkList& wl, std::vector<uint64_t>& acc,
-                std::vector<int32_t>& touched) {
+// Work items of one unit for one pass.  A unit is one owned head (w[0]
+// before batch replication) whose columns come from the adjacency rows of the
+// graph heads src_heads[j]: one for the query-owned pass, the query heads of
+// a K/V head's group for the key-owned pass (entries carry j).
+void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t unit,
+                const std::vector<int64_t>& src_heads, const std::vector<std::vector<int32_t>>& tiles, WorkList& wl,
+                std::vector<uint64_t>& acc, std::vector<int64_t>& touched) {
+  const int64_t npc = col.n_pages;
   const bool strided = strided_enabled();
   int32_t rg[kTilePages * kPageRows];
   for (const auto& tile : tiles) {
@@ -363,21 +380,22 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       const int s0 = it * kMaxSegments;
       const int s1 = std::min<int>(s0 + kMaxSegments, static_cast<int>(segs.size()));
       touched.clear();
-      for (int s = s0; s < s1; ++s) {
-        const int64_t r = static_cast<int64_t>(h) * adj.n_src + segs[s];
-        for (int64_t e = adj.ptr[r]; e < adj.ptr[r + 1]; ++e) {
-          const int32_t b = adj.dst[e];
-          for (int64_t x = col.gp_ptr[b]; x < col.gp_ptr[b + 1]; ++x) {
-            const int32_t p = col.gp_page[x];
-            if (acc[p] == 0) touched.push_back(p);
-            acc[p] |= static_cast<uint64_t>(col.gp_mask[x]) << (16 * (s - s0));
+      for (size_t j = 0; j < src_heads.size(); ++j)
+        for (int s = s0; s < s1; ++s) {
+          const int64_t r = src_heads[j] * adj.n_src + segs[s];
+          for (int64_t e = adj.ptr[r]; e < adj.ptr[r + 1]; ++e) {
+            const int32_t b = adj.dst[e];
+            for (int64_t x = col.gp_ptr[b]; x < col.gp_ptr[b + 1]; ++x) {
+              const int64_t c = static_cast<int64_t>(j) * npc + col.gp_page[x];  // (head offset, page)
+              if (acc[c] == 0) touched.push_back(c);
+              acc[c] |= static_cast<uint64_t>(col.gp_mask[x]) << (16 * (s - s0));
+            }
           }
         }
-      }
       std::sort(touched.begin(), touched.end());
       int32_t w[kWorkWords];
       std::memset(w, 0, sizeof(w));
-      w[0] = h;
+      w[0] = unit;
       w[1] = npg;
       w[2] = static_cast<int32_t>(wl.pages.size());
       // Column entries in slot order.  Up to four consecutive pages whose
@@ -389,12 +407,15 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       };
       size_t i = 0;
       while (i < touched.size()) {
-        const int32_t p = touched[i];
-        const int k = strided ? sub_group(fold(acc[p])) : -1;
+        const int64_t c = touched[i];
+        const int32_t p = static_cast<int32_t>(c % npc);
+        const uint16_t jh = static_cast<uint16_t>(c / npc);
+        const int k = strided ? sub_group(fold(acc[c])) : -1;
+        // (the bound keeps p + 3 inside the side, so c + 3 stays in head jh)
         if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= col.slots) {
           size_t j = i;
           bool same = true;
-          while (j < touched.size() && touched[j] <= p + 3) {
+          while (j < touched.size() && touched[j] <= c + 3) {
             if (sub_group(fold(acc[touched[j]])) != k) {
               same = false;
               break;
@@ -404,20 +425,22 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
           if (same && j - i >= 2) {
             uint64_t m = 0;
             for (size_t x = i; x < j; ++x) {
-              const int jj = touched[x] - p;
+              const int jj = static_cast<int>(touched[x] - c);
               for (int sg = 0; sg < kMaxSegments; ++sg)
                 m |= ((acc[touched[x]] >> (16 * sg + 4 * k)) & 0xFull) << (16 * sg + 4 * jj);
               acc[touched[x]] = 0;
             }
             wl.pages.push_back(~static_cast<int32_t>(16 * p + 4 * k));
             wl.masks.push_back(m);
+            wl.heads.push_back(jh);
             i = j;
             continue;
           }
         }
         wl.pages.push_back(p);
-        wl.masks.push_back(acc[p]);
-        acc[p] = 0;
+        wl.masks.push_back(acc[c]);
+        wl.heads.push_back(jh);
+        acc[c] = 0;
         ++i;
       }
       const size_t n_entries = wl.pages.size() - static_cast<size_t>(w[2]);
@@ -437,6 +460,56 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       wl.work.insert(wl.work.end(), w, w + kWorkWords);
     }
   }
+}
+
+// Work item templates of the slot-order tiles (the device planner's items):
+// the same rows, segments and row codes as build_head gives those tiles.
+void make_templates(const Side& own, PassTemplates& t) {
+  const auto tiles = pack_slot_order(owned_blocks(own));
+  t.words.clear();
+  t.segs.clear();
+  t.seg_rows.clear();
+  int32_t rg[kTilePages * kPageRows];
+  for (const auto& tile : tiles) {
+    const int npg = static_cast<int>(tile.size());
+    std::vector<int32_t> segs;
+    for (int r = 0; r < kTilePages * kPageRows; ++r) {
+      int32_t g = -2;
+      if (r < npg * kPageRows) {
+        const int64_t slot = pref_slot(tile[r / kPageRows], r % kPageRows);
+        if (slot < own.slots) g = own.group[slot];
+      }
+      rg[r] = g;
+      if (g >= 0 && std::find(segs.begin(), segs.end(), g) == segs.end()) segs.push_back(g);
+    }
+    const int n_items = std::max<int>(1, (static_cast<int>(segs.size()) + kMaxSegments - 1) / kMaxSegments);
+    for (int it = 0; it < n_items; ++it) {
+      const int s0 = it * kMaxSegments;
+      const int s1 = std::min<int>(s0 + kMaxSegments, static_cast<int>(segs.size()));
+      int32_t w[kWorkWords];
+      std::memset(w, 0, sizeof(w));
+      w[1] = npg;
+      for (int i = 0; i < npg; ++i) w[4 + i] = tile[i];
+      int32_t rows[kMaxSegments] = {0, 0, 0, 0};
+      for (int r = 0; r < kTilePages * kPageRows; ++r) {
+        uint32_t code = kCodeNotOwned;
+        if (rg[r] == -1) {
+          code = (it == 0) ? kCodeNoSegment : kCodeNotOwned;
+        } else if (rg[r] >= 0) {
+          for (int s = s0; s < s1; ++s)
+            if (segs[s] == rg[r]) code = static_cast<uint32_t>(s - s0);
+        }
+        if (code < 4) rows[code] += 1;
+        reinterpret_cast<uint32_t*>(w)[12 + r / 8] |= code << (4 * (r % 8));
+      }
+      t.words.insert(t.words.end(), w, w + kWorkWords);
+      for (int s = 0; s < kMaxSegments; ++s) {
+        t.segs.push_back(s0 + s < s1 ? segs[s0 + s] : -1);
+        t.seg_rows.push_back(rows[s]);
+      }
+    }
+  }
+  t.n = static_cast<int64_t>(t.words.size()) / kWorkWords;
 }
 
 // Items of one head, longest column list first: CTAs start in grid order,
@@ -467,36 +540,44 @@ int packing_mode() {
   return 0;
 }
 
-int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32_t heads, int32_t batch,
+// Work list of one pass.  Unit u (0 <= u < n_units) owns tensor head u of the
+// owned side (before batch replication) and takes its columns from the graph
+// heads src_heads(u); with one graph for every batch entry the units are the
+// heads of batch entry 0 and the items are repeated per batch entry with
+// their owned head shifted by b * owned_heads (they share the entries).
+int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32_t n_units, int32_t owned_heads,
+                   int32_t batch_copies, const std::function<std::vector<int64_t>(int32_t)>& src_heads,
                    WorkList& wl) {
   const auto blocks = owned_blocks(own);
   const auto slot_tiles = pack_slot_order(blocks);
 
   const int mode = packing_mode();
-  // Heads are independent: each is built on its own into part[h] (worker t
-  // takes heads t, t + n, ...), then the parts are joined in head order, so
+  // Units are independent: each is built on its own into part[u] (worker t
+  // takes units t, t + n, ...), then the parts are joined in unit order, so
   // the result does not depend on the number of threads.
-  std::vector<WorkList> part(heads);
+  std::vector<WorkList> part(n_units);
   // all hardware threads, unless SPATTN_PLAN_THREADS (>= 1) asks for fewer or more
   int want = static_cast<int>(std::thread::hardware_concurrency());
   if (const char* env = std::getenv("SPATTN_PLAN_THREADS")) want = std::max(1, std::atoi(env));
-  const int n_threads = std::max(1, std::min<int>(heads, want));
+  const int n_threads = std::max(1, std::min<int>(n_units, want));
   std::vector<char> failed(n_threads, 0);
   auto worker = [&](int t) {
     try {
-      std::vector<uint64_t> acc(col.n_pages, 0);
-      std::vector<int32_t> touched;
-      for (int32_t h = t; h < heads; h += n_threads) {
-        // Per head, the packing with fewer physical pairs (then fewer items).
-        if (mode != 2) build_head(own, col, adj, h, slot_tiles, part[h], acc, touched);
+      std::vector<int64_t> touched;
+      std::vector<uint64_t> acc;
+      for (int32_t u = t; u < n_units; u += n_threads) {
+        const std::vector<int64_t> src = src_heads(u);
+        acc.assign(static_cast<size_t>(col.n_pages) * src.size(), 0);
+        // Per unit, the packing with fewer physical pairs (then fewer items).
+        if (mode != 2) build_head(own, col, adj, u, src, slot_tiles, part[u], acc, touched);
         if (mode != 1) {
           WorkList sim;
-          build_head(own, col, adj, h, pack_similar(col, adj, h, blocks), sim, acc, touched);
-          const bool better = mode == 2 || sim.physical_pairs < part[h].physical_pairs ||
-                              (sim.physical_pairs == part[h].physical_pairs && sim.work.size() < part[h].work.size());
-          if (better) part[h] = std::move(sim);
+          build_head(own, col, adj, u, src, pack_similar(col, adj, src, blocks), sim, acc, touched);
+          const bool better = mode == 2 || sim.physical_pairs < part[u].physical_pairs ||
+                              (sim.physical_pairs == part[u].physical_pairs && sim.work.size() < part[u].work.size());
+          if (better) part[u] = std::move(sim);
         }
-        order_longest_first(part[h]);
+        order_longest_first(part[u]);
       }
     } catch (...) {
       failed[t] = 1;  // an allocation failed; reported below as OOM
@@ -526,9 +607,11 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   wl.work.clear();
   wl.pages.clear();
   wl.masks.clear();
+  wl.heads.clear();
   wl.physical_pairs = 0;
   wl.pages.reserve(n_entries);
   wl.masks.reserve(n_entries);
+  wl.heads.reserve(n_entries);
   for (auto& pt : part) {
     const int32_t off = static_cast<int32_t>(wl.pages.size());  // entry ranges are per part
     for (size_t i = 0; i < pt.work.size(); i += kWorkWords) {
@@ -538,22 +621,25 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
     wl.work.insert(wl.work.end(), pt.work.begin(), pt.work.end());
     wl.pages.insert(wl.pages.end(), pt.pages.begin(), pt.pages.end());
     wl.masks.insert(wl.masks.end(), pt.masks.begin(), pt.masks.end());
+    wl.heads.insert(wl.heads.end(), pt.heads.begin(), pt.heads.end());
     wl.physical_pairs += pt.physical_pairs;
     pt = WorkList();  // release the part's memory as soon as it is copied
   }
-  const int64_t per_batch = static_cast<int64_t>(wl.work.size()) / kWorkWords;
+  const int64_t per_copy = static_cast<int64_t>(wl.work.size()) / kWorkWords;
   std::vector<int32_t> all;
-  all.reserve(static_cast<size_t>(per_batch) * batch * kWorkWords);
-  for (int32_t b = 0; b < batch; ++b)
-    for (int64_t i = 0; i < per_batch; ++i) {
+  all.reserve(static_cast<size_t>(per_copy) * batch_copies * kWorkWords);
+  for (int32_t b = 0; b < batch_copies; ++b)
+    for (int64_t i = 0; i < per_copy; ++i) {
       const int32_t* w = wl.work.data() + i * kWorkWords;
       all.insert(all.end(), w, w + kWorkWords);
-      all[all.size() - kWorkWords] = b * heads + w[0];
+      all[all.size() - kWorkWords] = b * owned_heads + w[0];
     }
   wl.work.swap(all);
-  wl.n_work = per_batch * batch;
+  wl.n_work = per_copy * batch_copies;
+  wl.physical_pairs *= batch_copies;
   return SPATTN_OK;
 }
+
 
 // Rows of one side that no work item writes, as (page, row mask) pairs:
 // pages without a valid slot (all 16 rows), and the rows outside the 4-row
@@ -576,9 +662,10 @@ void fill_list(const Side& s, std::vector<int32_t>& out) {
 }
 
 template <typename T>
-int upload(const std::vector<T>& host, T** dev, int64_t& bytes) {
+int upload(const std::vector<T>& host, T** dev, int64_t& bytes, int64_t* cap = nullptr) {
   const size_t n = std::max<size_t>(host.size(), 1) * sizeof(T);
   if (cudaMalloc(reinterpret_cast<void**>(dev), n) != cudaSuccess) return SPATTN_ERR_OOM;
+  if (cap) *cap = static_cast<int64_t>(std::max<size_t>(host.size(), 1));
   bytes += static_cast<int64_t>(n);
   if (!host.empty() && cudaMemcpy(*dev, host.data(), host.size() * sizeof(T), cudaMemcpyHostToDevice) != cudaSuccess)
     return SPATTN_ERR_CUDA;
@@ -632,7 +719,7 @@ int64_t bsa_pairs(const spattn_plan_s& P) {
   const int per = kBlockRows / kPageRows;
   std::vector<int32_t> pages;
   int64_t count = 0;
-  for (int32_t h = 0; h < P.heads; ++h)
+  for (int32_t h = 0; h < P.graph_batches * P.heads; ++h)
     for (int64_t qb = 0; qb < n_qb; ++qb) {
       canonical_pages(P, h, qb, pages);
       int64_t prev = -1;
@@ -642,10 +729,15 @@ int64_t bsa_pairs(const spattn_plan_s& P) {
           ++count;
         }
     }
-  return count * kBlockRows * kBlockRows * P.batch;
+  return count * kBlockRows * kBlockRows * (P.batch / P.graph_batches);
 }
 
+void free_device_planner(DevPlanner& d);
+
 void free_plan_device(spattn_plan_s* P) {
+  free_device_planner(P->dp);
+  cudaFree(P->wk.d_heads);
+  P->wk.d_heads = nullptr;
   cudaFree(P->wq.d_work);
   cudaFree(P->wq.d_pages);
   cudaFree(P->wq.d_masks);
@@ -664,6 +756,39 @@ void free_plan_device(spattn_plan_s* P) {
   P->n_events = 0;
 }
 
+// After a device re-plan: bring the work lists and the graph back to the host
+// copies that the inspection calls read (synchronises the device).
+int refresh_host(spattn_plan_s* P) {
+  if (!P->host_stale) return SPATTN_OK;
+  if (cudaDeviceSynchronize() != cudaSuccess) return SPATTN_ERR_CUDA;
+  for (WorkList* w : {&P->wq, &P->wk}) {
+    w->work.resize(static_cast<size_t>(w->n_work) * kWorkWords);
+    w->pages.resize(static_cast<size_t>(w->n_entries_dev));
+    w->masks.resize(static_cast<size_t>(w->n_entries_dev));
+    if ((!w->work.empty() && cudaMemcpy(w->work.data(), w->d_work, w->work.size() * sizeof(int32_t),
+                                        cudaMemcpyDeviceToHost) != cudaSuccess) ||
+        (!w->pages.empty() && cudaMemcpy(w->pages.data(), w->d_pages, w->pages.size() * sizeof(int32_t),
+                                         cudaMemcpyDeviceToHost) != cudaSuccess) ||
+        (!w->masks.empty() && cudaMemcpy(w->masks.data(), w->d_masks, w->masks.size() * sizeof(uint64_t),
+                                         cudaMemcpyDeviceToHost) != cudaSuccess))
+      return SPATTN_ERR_CUDA;
+  }
+  const int64_t rows = static_cast<int64_t>(P->graph_batches) * P->heads * P->q.n_groups;
+  std::vector<int64_t> rp(rows + 1);
+  std::vector<int32_t> dst(std::max<int64_t>(P->graph_nnz, 1));
+  if (cudaMemcpy(rp.data(), P->dp.d_fwd_ptr, rp.size() * sizeof(int64_t), cudaMemcpyDeviceToHost) != cudaSuccess ||
+      (P->graph_nnz > 0 && cudaMemcpy(dst.data(), P->dp.d_fwd_dst, P->graph_nnz * sizeof(int32_t),
+                                      cudaMemcpyDeviceToHost) != cudaSuccess))
+    return SPATTN_ERR_CUDA;
+  spattn_graph g{rp.data(), dst.data()};
+  const int32_t GH = P->graph_batches * P->heads;
+  int st = build_fwd_adjacency(&g, GH, P->q.n_groups, P->k.n_groups, P->fwd_adj);
+  if (st) return st;
+  build_bwd_adjacency(P->fwd_adj, GH, P->q.n_groups, P->k.n_groups, P->bwd_adj);
+  P->host_stale = false;
+  return SPATTN_OK;
+}
+
 int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) {
   const auto t0 = std::chrono::steady_clock::now();
   if (!L || !G || !L->q_group || !L->kv_group || !G->row_ptr) return SPATTN_ERR_INVALID_ARG;
@@ -673,10 +798,20 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if (L->q_slots >= (int64_t(1) << 31) - 64 || L->kv_slots >= (int64_t(1) << 31) - 64) return SPATTN_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(L->batch) * L->heads >= (int64_t(1) << 31)) return SPATTN_ERR_UNSUPPORTED;
   if (!std::isfinite(L->scale) || L->scale < 0.f) return SPATTN_ERR_INVALID_ARG;
-  if (G->row_ptr[static_cast<int64_t>(L->heads) * L->n_q_groups] > 0 && !G->kv_groups) return SPATTN_ERR_INVALID_ARG;
+  const int32_t kv_heads = L->kv_heads == 0 ? L->heads : L->kv_heads;
+  if (kv_heads < 1 || L->heads % kv_heads != 0) return SPATTN_ERR_INVALID_ARG;
+  if (L->heads / kv_heads > 65535) return SPATTN_ERR_UNSUPPORTED;
+  const int32_t gb = L->graph_batches == 0 ? 1 : L->graph_batches;
+  if (gb != 1 && gb != L->batch) return SPATTN_ERR_INVALID_ARG;
+  const int32_t GH = gb * L->heads;  // graph heads: one graph per (graph batch, head)
+  if (static_cast<int64_t>(GH) * std::max(L->n_q_groups, L->n_kv_groups) >= (int64_t(1) << 40))
+    return SPATTN_ERR_UNSUPPORTED;
+  if (G->row_ptr[static_cast<int64_t>(GH) * L->n_q_groups] > 0 && !G->kv_groups) return SPATTN_ERR_INVALID_ARG;
 
   P->batch = L->batch;
   P->heads = L->heads;
+  P->kv_heads = kv_heads;
+  P->graph_batches = gb;
   P->head_dim = L->head_dim;
   P->scale = L->scale != 0.f ? L->scale : 1.0f / std::sqrt(static_cast<float>(L->head_dim));
   // Without a usable CUDA device the plan is kept on the host only: the
@@ -691,38 +826,54 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if (st) return st;
   st = build_side(L->kv_slots, L->kv_group, L->n_kv_groups, P->k);
   if (st) return st;
-  st = build_fwd_adjacency(G, L->heads, L->n_q_groups, L->n_kv_groups, P->fwd_adj);
+  st = build_fwd_adjacency(G, GH, L->n_q_groups, L->n_kv_groups, P->fwd_adj);
   if (st) return st;
-  build_bwd_adjacency(P->fwd_adj, L->heads, L->n_q_groups, L->n_kv_groups, P->bwd_adj);
+  build_bwd_adjacency(P->fwd_adj, GH, L->n_q_groups, L->n_kv_groups, P->bwd_adj);
 
   int64_t useful = 0;
-  for (int32_t h = 0; h < L->heads; ++h)
+  for (int32_t h = 0; h < GH; ++h)
     for (int32_t a = 0; a < L->n_q_groups; ++a) {
       const int64_t r = static_cast<int64_t>(h) * L->n_q_groups + a;
       int64_t nk = 0;
       for (int64_t e = P->fwd_adj.ptr[r]; e < P->fwd_adj.ptr[r + 1]; ++e) nk += P->k.group_size[P->fwd_adj.dst[e]];
       useful += P->q.group_size[a] * nk;
     }
-  P->useful_pairs = useful * L->batch;
+  const int32_t copies = L->batch / gb;  // batch entries that share each graph
+  P->useful_pairs = useful * copies;
 
-  st = build_worklist(P->q, P->k, P->fwd_adj, L->heads, L->batch, P->wq);
+  // query-owned pass: unit = graph head (its own graph rows)
+  st = build_worklist(P->q, P->k, P->fwd_adj, GH, L->heads, copies,
+                      [](int32_t u) { return std::vector<int64_t>{u}; }, P->wq);
   if (st) return st;
-  st = build_worklist(P->k, P->q, P->bwd_adj, L->heads, L->batch, P->wk);
+  // key-owned pass: unit = K/V head of a graph batch; its columns are the
+  // transposed rows of the query heads of its group (head offset j)
+  const int32_t grp = L->heads / kv_heads;
+  const int32_t H = L->heads;
+  st = build_worklist(P->k, P->q, P->bwd_adj, gb * kv_heads, kv_heads, copies,
+                      [=](int32_t u) {
+                        std::vector<int64_t> v(grp);
+                        for (int32_t j = 0; j < grp; ++j)
+                          v[j] = static_cast<int64_t>(u / kv_heads) * H + (u % kv_heads) * grp + j;
+                        return v;
+                      },
+                      P->wk);
   if (st) return st;
 
   fill_list(P->q, P->q_fill);
   fill_list(P->k, P->k_fill);
+  make_templates(P->q, P->dp.tq);
+  make_templates(P->k, P->dp.tk);
 
   P->plan_ms = std::chrono::duration<double, std::milli>(std::chrono::steady_clock::now() - t0).count();
   if (P->device < 0) return SPATTN_OK;
 
   int64_t bytes = 0;
-  if ((st = upload(P->wq.work, &P->wq.d_work, bytes))) return st;
-  if ((st = upload(P->wq.pages, &P->wq.d_pages, bytes))) return st;
-  if ((st = upload(P->wq.masks, &P->wq.d_masks, bytes))) return st;
-  if ((st = upload(P->wk.work, &P->wk.d_work, bytes))) return st;
-  if ((st = upload(P->wk.pages, &P->wk.d_pages, bytes))) return st;
-  if ((st = upload(P->wk.masks, &P->wk.d_masks, bytes))) return st;
+  if ((st = upload(P->wk.heads, &P->wk.d_heads, bytes))) return st;
+  for (WorkList* w : {&P->wq, &P->wk}) {
+    if ((st = upload(w->work, &w->d_work, bytes, &w->cap_work))) return st;
+    if ((st = upload(w->pages, &w->d_pages, bytes, &w->cap_pages))) return st;
+    if ((st = upload(w->masks, &w->d_masks, bytes, &w->cap_masks))) return st;
+  }
   if ((st = upload(P->q_fill, &P->d_q_fill, bytes))) return st;
   if ((st = upload(P->k_fill, &P->d_k_fill, bytes))) return st;
   if (cudaMalloc(reinterpret_cast<void**>(&P->d_err), sizeof(int)) != cudaSuccess) return SPATTN_ERR_OOM;

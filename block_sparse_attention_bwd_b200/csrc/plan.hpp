@@ -60,17 +60,62 @@ struct WorkList {
   std::vector<int32_t> work;     // n_work * kWorkWords (all batches)
   std::vector<int32_t> pages;    // entries of one batch
   std::vector<uint64_t> masks;
+  // per entry: the query head of the entry within the item's K/V head group
+  // (key-owned pass under grouped-query attention; 0 otherwise)
+  std::vector<uint16_t> heads;
+  uint16_t* d_heads = nullptr;
   int64_t n_work = 0;
   int64_t physical_pairs = 0;    // one batch
   int32_t* d_work = nullptr;
   int32_t* d_pages = nullptr;
   uint64_t* d_masks = nullptr;
+  // capacities of the device arrays (elements) and, after a device re-plan,
+  // the number of entries on the device
+  int64_t cap_work = 0, cap_pages = 0, cap_masks = 0;
+  int64_t n_entries_dev = -1;
 };
+
+// Work item templates of one pass for the device planner: the slot-order
+// tiles of the layout split into items, without their column lists.
+struct PassTemplates {
+  std::vector<int32_t> words;     // n x kWorkWords (bh and entry range set on the device)
+  std::vector<int32_t> segs;      // n x 4 group of each segment, -1 = none
+  std::vector<int32_t> seg_rows;  // n x 4 owned rows of each segment
+  int64_t n = 0;
+  int32_t* d_words = nullptr;
+  int32_t* d_segs = nullptr;
+  int32_t* d_seg_rows = nullptr;
+};
+
+// Device state of spattn_plan_set_graph_device (allocated on first use).
+struct DevPlanner {
+  bool ready = false;
+  PassTemplates tq, tk;  // query-owned, key-owned
+  int64_t* d_q_gp_ptr = nullptr;
+  int32_t* d_q_gp_page = nullptr;
+  uint16_t* d_q_gp_mask = nullptr;
+  int64_t* d_k_gp_ptr = nullptr;
+  int32_t* d_k_gp_page = nullptr;
+  uint16_t* d_k_gp_mask = nullptr;
+  int64_t* d_fwd_ptr = nullptr;   // the graph (plan-owned copy)
+  int32_t* d_fwd_dst = nullptr;
+  int64_t fwd_cap = 0;
+  int64_t* d_bwd_ptr = nullptr;   // its transpose
+  int32_t* d_bwd_dst = nullptr;
+  int64_t bwd_cap = 0;
+  int64_t* d_cursor = nullptr;
+  int64_t* d_counts = nullptr;
+  unsigned long long* d_stats = nullptr;
+};
+
+bool strided_setting();
 
 }  // namespace spattn
 
 struct spattn_plan_s {
   int32_t batch = 0, heads = 0, head_dim = 0;
+  int32_t kv_heads = 0;       // K/V heads (heads % kv_heads == 0)
+  int32_t graph_batches = 1;  // 1: one graph for every batch entry; batch: one graph per entry
   float scale = 0.f;
   int device = 0;
   spattn::Side q, k;
@@ -87,6 +132,9 @@ struct spattn_plan_s {
   int32_t* d_k_fill = nullptr;
   int* d_err = nullptr;        // device error word
   float* d_delta = nullptr;    // [batch, heads, q_slots] rowsum(dO * O)
+  spattn::DevPlanner dp;        // device planner state
+  bool host_stale = false;      // the work lists / graph were rebuilt on the device
+  int64_t graph_nnz = 0;        // entries of the graph the device lists follow
   int64_t useful_pairs = 0;
   int64_t bsa_pairs = -1;      // computed on first request
   int64_t device_bytes = 0;

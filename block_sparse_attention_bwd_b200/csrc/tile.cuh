@@ -71,7 +71,8 @@ struct StepMasks {
 
 // Warp-collective TMA gather of n (<= 32) pages into a stage whose 64-column
 // chunks are `chunk_bytes` apart; page j lands at rows 16j..16j+15 of every
-// chunk.  Lane j < n holds page id `pid` of page j.  Maximal runs of
+// chunk.  Lane j < n holds page id `pid` of page j and the batch*head `bh` it
+// is read from (a run never spans two heads).  Maximal runs of
 // consecutive page ids are fetched with 64-, 32- and 16-row boxes by the
 // run's first lane; a run that fills a whole 64-row stage (chunks 8 KB
 // apart) or a whole 128-row stage or tile (chunks 16 KB apart) takes one
@@ -86,8 +87,9 @@ __device__ __forceinline__ void load_page_runs(uint8_t* dst, int chunk_bytes, co
                                                int bh, uint64_t* bar) {
   const int lane = lane_id();
   const int nxt = __shfl_down_sync(0xffffffffu, pid, 1);
-  // bit j: page j+1 follows page j (both regular)
-  const unsigned cont = __ballot_sync(0xffffffffu, lane + 1 < n && pid >= 0 && nxt == pid + 1);
+  const int nbh = __shfl_down_sync(0xffffffffu, bh, 1);
+  // bit j: page j+1 follows page j (both regular, same batch*head)
+  const unsigned cont = __ballot_sync(0xffffffffu, lane + 1 < n && pid >= 0 && nxt == pid + 1 && nbh == bh);
   const bool start = lane < n && (lane == 0 || !((cont >> (lane - 1)) & 1u));
   if (!start) return;
   if (pid < 0) {

@@ -19,7 +19,9 @@
  *   - The graph is a CSR over (head, query group): entries
  *     kv_groups[row_ptr[r] .. row_ptr[r+1]) with r = head * n_q_groups + a
  *     are the key groups that query group a may attend in that head.  The
- *     same graph serves every batch index.  Duplicate entries are allowed.
+ *     same graph serves every batch index, unless layout.graph_batches =
+ *     batch: then row r = (b * heads + head) * n_q_groups + a holds batch
+ *     entry b's graph.  Duplicate entries are allowed.
  *   - Query slot i may attend key slot j in head h iff both are valid and
  *     kv_group[j] is listed for q_group[i].
  *   - A page is 16 consecutive slots; a Q block is 64 consecutive query
@@ -27,7 +29,9 @@
  *
  * Tensors (all device pointers, owned by the caller)
  *   Q, O, dO, dQ : bf16 [batch, heads, q_slots, head_dim], contiguous
- *   K, V, dK, dV : bf16 [batch, heads, kv_slots, head_dim], contiguous
+ *   K, V, dK, dV : bf16 [batch, kv_heads, kv_slots, head_dim], contiguous
+ *                  (dK, dV of a K/V head sum the gradients of all query
+ *                  heads that read it)
  *   LSE          : fp32 [batch, heads, q_slots], natural log of
  *                  sum_j exp(scale * q_i . k_j) over the allowed keys.
  *   Every pointer must be 16-byte aligned.  head_dim is 64 or 128.
@@ -70,6 +74,12 @@ typedef struct {
   const int32_t* kv_group;        /* host [kv_slots], -1 = padded */
   int32_t n_q_groups, n_kv_groups;
   float scale;                    /* softmax scale > 0; 0 selects 1/sqrt(head_dim) */
+  int32_t kv_heads;               /* K/V heads for grouped-query attention: heads % kv_heads == 0,
+                                     query head h reads K/V head h / (heads / kv_heads);
+                                     0 selects kv_heads = heads (1 = multi-query) */
+  int32_t graph_batches;          /* 0 or 1: one graph for every batch entry; batch: one graph per
+                                     batch entry (the graph then has batch * heads * n_q_groups rows,
+                                     batch-major) */
 } spattn_layout;
 
 typedef struct {
@@ -129,6 +139,27 @@ int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_p
  * that computes fewer physical pairs; SPATTN_PLAN_PACK=slot or =similar
  * forces one of them.  Work items of a head run longest column list
  * first.) */
+
+/* Re-plan for a new sparse graph over the plan's layout, on the GPU.
+ * Dynamic block selection (VSA-style graphs, one of the layouts the KPage
+ * abstract evaluates, zhuanzhiai.com paper page) changes the graph every
+ * call, and host planning of a large graph takes about a second; this call
+ * rebuilds both work lists on the device in milliseconds.  row_ptr
+ * ([heads * n_q_groups + 1]) and kv_groups ([nnz]) are DEVICE arrays in the
+ * format of spattn_graph (rows may be unsorted and hold duplicates), read on
+ * `stream`; the plan keeps its own copy.  The owned tiles are the layout's
+ * slot-order tiles (with strided pages); the column lists, strided entries,
+ * pair counts and the transposed (key-owned) lists follow the new graph and
+ * are identical to what spattn_plan would build with SPATTN_PLAN_PACK=slot,
+ * up to the order of the work items.  The call synchronises `stream` once;
+ * the new lists are used by every later spattn_fwd / spattn_bwd.  Returns
+ * SPATTN_ERR_INVALID_ARG for a malformed graph (the plan is left unchanged),
+ * SPATTN_ERR_UNSUPPORTED if one work item would gather more than 8192
+ * (page, group) pairs, SPATTN_ERR_OOM if growing the plan's device lists
+ * fails.  The inspection calls (stats, pages, qblocks, work) describe the
+ * new graph (their first call copies it back to the host). */
+int spattn_plan_set_graph_device(spattn_plan_t plan, const int64_t* row_ptr, const int32_t* kv_groups, int64_t nnz,
+                                 void* stream);
 
 /* Forward: O and LSE for every query slot of every (batch, head): masked
  * softmax attention over exactly the plan's sparse graph, computed over the
@@ -194,6 +225,8 @@ int spattn_plan_stats(spattn_plan_t plan, spattn_stats* stats);
 int spattn_profile(spattn_plan_t plan, int enable);
 int spattn_profile_read(spattn_plan_t plan, spattn_kernel_times* out);
 
+/* In spattn_plan_pages and spattn_plan_qblocks, `head` is a graph head:
+ * b * heads + h when each batch entry has its own graph, else h. */
 /* Canonical page list of (head, Q block): ascending pages holding at least
  * one key that some query of the block may attend (the 16-row K/V pages a Q
  * block needs; KPage abstract, zhuanzhiai.com paper page).  *pages points into a
@@ -208,7 +241,8 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
 /* Host copy of a work list, for inspection and tests (the packed tiles of
  * the KPage abstract's load-time packing, zhuanzhiai.com paper page).  which = 0: query-owned
  * (forward and dQ), 1: key-owned (dK/dV).  Each work item is 32 int32 words:
- *   [0] batch*heads + head   [1] owned page count n (<= 8)
+ *   [0] batch*heads + head of the owned side (query heads for which = 0,
+ *       K/V heads for which = 1)   [1] owned page count n (<= 8)
  *   [2] first entry          [3] end entry (into pages/masks)
  *   [4..11] owned page ids   [12..27] 128 row codes, 4 bits each, row r in
  *   word 12 + r/8 at bit 4*(r%8): 0..3 = segment, 14 = owned row with no
@@ -218,6 +252,12 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
  * Entries are shared by all batch indices. */
 int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work,
                      const int32_t** pages, const uint64_t** masks, int64_t* n_entries);
+
+/* Per entry of work list `which` (as in spattn_plan_work): the query head of
+ * the entry relative to the first query head of the item's K/V head (always
+ * 0 for the query-owned list and without grouped-query attention); the
+ * array has the same length and buffer rules as spattn_plan_work's. */
+int spattn_plan_entry_heads(spattn_plan_t plan, int32_t which, const uint16_t** heads, int64_t* n_entries);
 
 /* Free the plan and its device lists (NULL is a no-op).  The caller must
  * make sure no kernel launched with the plan is still running.  (Plan

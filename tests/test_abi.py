@@ -123,3 +123,19 @@ def sp_device_available():
         return torch.cuda.is_available()
     except Exception:
         return False
+
+
+def test_device_replan_needs_a_device_and_arguments():
+    """spattn_plan_set_graph_device: argument checks on the host, and a plan
+    built without a device answers SPATTN_ERR_CUDA."""
+    p = W.make_problem("tiny")
+    pl = _plan(p)
+    lib = sp.load_library()
+    one = ctypes.c_void_p(16)
+    assert lib.spattn_plan_set_graph_device(None, one, one, 0, None) == sp.SPATTN_ERR_INVALID_ARG
+    assert lib.spattn_plan_set_graph_device(pl.handle, None, one, 0, None) == sp.SPATTN_ERR_INVALID_ARG
+    assert lib.spattn_plan_set_graph_device(pl.handle, one, None, 5, None) == sp.SPATTN_ERR_INVALID_ARG
+    assert lib.spattn_plan_set_graph_device(pl.handle, one, one, -1, None) == sp.SPATTN_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.spattn_plan_set_graph_device(pl.handle, one, one, 0, None) == sp.SPATTN_ERR_CUDA

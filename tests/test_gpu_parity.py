@@ -73,15 +73,23 @@ def check_padded(p, out):
 
 
 def check_tiny(p, t, out, batch):
-    """Full comparison of every (batch, head); returns the pooled arrays."""
+    """Full comparison of every (batch, head).  Under grouped-query attention
+    a query head h reads K/V head h // (heads / kv_heads), and dK, dV of a
+    K/V head are the sums over its query heads; with one graph per batch
+    entry, (b, h) uses the graph of graph head b * heads + h."""
     check_padded(p, out)
     vq = p.q_group >= 0
     vk = p.kv_group >= 0
+    H, Hkv = p.heads, p.n_kv_heads
+    grp = H // Hkv
     pooled = {k: ([], []) for k in ("o", "dq", "dk", "dv")}
+    kv_ref = {}
     for b in range(batch):
-        for h in range(p.heads):
-            A = _allowed(p, h)
-            q, k, v, do = (_f64(t[n][b, h]) for n in ("q", "k", "v", "do"))
+        for h in range(H):
+            hk = h // grp
+            A = _allowed(p, p.graph_head(b, h))
+            q, do = _f64(t["q"][b, h]), _f64(t["do"][b, h])
+            k, v = _f64(t["k"][b, hk]), _f64(t["v"][b, hk])
             M = oracle.token_mask(p.q_group, p.kv_group, A)
             o_ref, lse_ref = oracle.forward(q, k, v, M, p.scale)
             dq_ref, dk_ref, dv_ref = oracle.backward(q, k, v, do, M, p.scale)
@@ -93,24 +101,31 @@ def check_tiny(p, t, out, batch):
             assert np.abs(o_g[vq] - o_ref[vq]).max() <= TOL["o_abs"], (b, h)
             assert rel_l2(o_g[vq], o_ref[vq]) <= TOL["o_rel"], (b, h, rel_l2(o_g[vq], o_ref[vq]))
             pooled["o"][0].append(o_g[vq]); pooled["o"][1].append(o_ref[vq])
-            for name, ref, valid in (("dq", dq_ref, vq), ("dk", dk_ref, vk), ("dv", dv_ref, vk)):
-                g = _f64(out[name][b, h])[valid]
-                r = ref[valid]
-                assert rel_l2(g, r) <= TOL["grad_rel"], (name, b, h, rel_l2(g, r))
-                pooled[name][0].append(g); pooled[name][1].append(r)
-            # attention-free valid rows are exact zeros; keys nobody attends get exact zero gradients
+            dq_g = _f64(out["dq"][b, h])
+            assert rel_l2(dq_g[vq], dq_ref[vq]) <= TOL["grad_rel"], ("dq", b, h, rel_l2(dq_g[vq], dq_ref[vq]))
+            pooled["dq"][0].append(dq_g[vq]); pooled["dq"][1].append(dq_ref[vq])
+            # attention-free valid rows are exact zeros
             assert np.all(o_g[~nonempty] == 0)
-            assert np.all(_f64(out["dq"][b, h])[~nonempty] == 0)
-            unreached = ~M.any(axis=0)
-            assert np.all(_f64(out["dk"][b, h])[unreached] == 0)
-            assert np.all(_f64(out["dv"][b, h])[unreached] == 0)
+            assert np.all(dq_g[~nonempty] == 0)
+            acc = kv_ref.setdefault((b, hk), [0.0, 0.0, np.zeros(p.kv_slots, bool)])
+            acc[0] = acc[0] + dk_ref
+            acc[1] = acc[1] + dv_ref
+            acc[2] |= M.any(axis=0)
+    for (b, hk), (dk_ref, dv_ref, reached) in kv_ref.items():
+        for name, ref in (("dk", dk_ref), ("dv", dv_ref)):
+            g = _f64(out[name][b, hk])
+            assert rel_l2(g[vk], ref[vk]) <= TOL["grad_rel"], (name, b, hk, rel_l2(g[vk], ref[vk]))
+            pooled[name][0].append(g[vk]); pooled[name][1].append(ref[vk])
+            # keys no query head of the group attends get exact zero gradients
+            assert np.all(g[~reached] == 0), (name, b, hk)
     g = {k: (np.concatenate(a), np.concatenate(r)) for k, (a, r) in pooled.items() if a}
     assert rel_l2(*g["o"]) <= TOL["o_rel"], rel_l2(*g["o"])
     for k in ("dq", "dk", "dv"):
         assert rel_l2(*g[k]) <= TOL["grad_rel"], (k, rel_l2(*g[k]))
 
 
-@pytest.mark.parametrize("name,batch", [(n, 1) for n in ["tiny"] + list(W.EXTRA_TINY)] + [("tiny_svg2", 2)])
+@pytest.mark.parametrize("name,batch", [(n, 1) for n in ["tiny"] + list(W.EXTRA_TINY) if n != "tiny_bgraph"]
+                         + [("tiny_svg2", 2), ("tiny_gqa", 2), ("tiny_bgraph", 2)])
 def test_tiny_full_parity(name, batch):
     p = W.make_problem(name)
     t, out, _ = run_gpu(p, batch=batch)

@@ -221,3 +221,65 @@ def test_strided_pages_stay_inside_the_tensor():
     pairs, _ = _covered(W.Problem("ragged", 1, 1, 64, qg, kg, 1, 1, np.array([0, 1], np.int64),
                                   np.array([0], np.int32), 0), pl, 0)
     assert sorted(j for (_, _, j) in pairs) == sorted(np.nonzero(kg >= 0)[0].tolist() * 16)
+
+
+def _covered_heads(p, pl, which, batch):
+    """{(owned bh, owned slot, column bh, column slot): count} over all work
+    items, with the column head of key-owned entries resolved through the
+    entry head offsets (grouped-query attention)."""
+    work, pages, masks = pl.work(which)
+    eh = pl.entry_heads(which)
+    H, Hkv = p.heads, p.n_kv_heads
+    g = H // Hkv
+    out = {}
+    bits16 = np.arange(16, dtype=np.uint64)
+    for w in work:
+        bh = int(w[0])
+        codes = _codes(w)
+        e0, e1 = int(w[2]), int(w[3])
+        col_slot = [pref_slots(x) for x in pages[e0:e1]]
+        for r in range(128):
+            c = int(codes[r])
+            if c >= 14:
+                continue
+            slot = int(pref_slots(w[4 + r // 16])[r % 16])
+            for e in range(e0, e1):
+                m = (int(masks[e]) >> (16 * c)) & 0xFFFF
+                if not m:
+                    continue
+                cbh = bh if which == 0 else (bh // Hkv) * H + (bh % Hkv) * g + int(eh[e])
+                if which == 0:
+                    cbh = (bh // H) * Hkv + (bh % H) // g
+                for bit in range(16):
+                    if (m >> bit) & 1:
+                        key = (bh, slot, cbh, int(col_slot[e - e0][bit]))
+                        out[key] = out.get(key, 0) + 1
+    return out
+
+
+@pytest.mark.parametrize("name", ["tiny_gqa", "tiny_mqa", "tiny_bgraph"])
+def test_coverage_grouped_heads_and_batch_graphs(name):
+    """Grouped-query attention and per-batch graphs: the query-owned list
+    computes, for every (batch, query head), exactly the pairs of that head's
+    graph against its K/V head; the key-owned list computes, for every
+    (batch, K/V head), the pairs of all query heads of its group, each once."""
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p)
+    B, H, Hkv = p.batch, p.heads, p.n_kv_heads
+    g = H // Hkv
+    expect_q, expect_k = set(), set()
+    for b in range(B):
+        for h in range(H):
+            A = _allowed(p, p.graph_head(b, h))
+            M = oracle.token_mask(p.q_group, p.kv_group, A)
+            hk = h // g
+            for i, j in zip(*np.nonzero(M)):
+                expect_q.add((b * H + h, int(i), b * Hkv + hk, int(j)))
+                expect_k.add((b * Hkv + hk, int(j), b * H + h, int(i)))
+    got_q = _covered_heads(p, pl, 0, B)
+    got_k = _covered_heads(p, pl, 1, B)
+    assert all(v == 1 for v in got_q.values()) and all(v == 1 for v in got_k.values())
+    assert set(got_q) == expect_q
+    assert set(got_k) == expect_k
+    st = pl.stats()
+    assert st["useful_pairs"] == len(expect_q)

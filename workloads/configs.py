@@ -57,7 +57,8 @@ import numpy as np
 PAD_SENTINEL = 1000.0
 
 CONFIG_NAMES = ("tiny", "full", "partial", "vsa", "svg2")
-EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_nokeys", "tiny_hedge")
+EXTRA_TINY = ("tiny_vsa", "tiny_svg2", "tiny_empty", "tiny_d128", "tiny_onekey", "tiny_nokeys", "tiny_hedge",
+              "tiny_gqa", "tiny_mqa", "tiny_bgraph")
 
 
 @dataclasses.dataclass
@@ -74,6 +75,16 @@ class Problem:
     kv_groups: np.ndarray  # int32 [nnz]
     seed_base: int
     description: str = ""
+    kv_heads: int = 0        # K/V heads (grouped-query attention); 0 = heads
+    graph_batches: int = 1   # 1: one graph for every batch entry; batch: one graph per entry
+
+    @property
+    def n_kv_heads(self) -> int:
+        return self.heads if self.kv_heads == 0 else self.kv_heads
+
+    def graph_head(self, b: int, h: int) -> int:
+        """Row block of the graph that (batch entry b, query head h) uses."""
+        return (b * self.heads + h) if self.graph_batches > 1 else h
 
     @property
     def q_slots(self) -> int:
@@ -261,6 +272,24 @@ def make_problem(name: str) -> Problem:
         row_ptr, cols = sta_graph(tiles, (1, 2, 2), 2)
         return Problem(name, 1, 2, 64, group, group.copy(), 6, 6, row_ptr, cols, 16000,
                        "tiny STA whose H-edge tiles keep one dh row (strided pages)")
+    if name in ("tiny_gqa", "tiny_mqa"):
+        # grouped-query attention: 4 query heads over 2 K/V heads (gqa) or 3
+        # over 1 (mqa); every query head has its own VSA-style lists
+        heads, kvh = (4, 2) if name == "tiny_gqa" else (3, 1)
+        group, tiles = sta_layout((5, 6, 10))
+        rng = np.random.default_rng(17005 if name == "tiny_gqa" else 18005)
+        row_ptr, cols = vsa_graph(12, heads, 4, rng)
+        return Problem(name, 1, heads, 64, group, group.copy(), 12, 12, row_ptr, cols,
+                       17000 if name == "tiny_gqa" else 18000,
+                       f"tiny VSA-style, {heads} query heads over {kvh} K/V head(s)", kv_heads=kvh)
+    if name == "tiny_bgraph":
+        # two batch entries with their own graphs (own tile + 3 random tiles
+        # per query tile, drawn per batch entry and head)
+        group, tiles = sta_layout((5, 6, 10))
+        rng = np.random.default_rng(19005)
+        row_ptr, cols = vsa_graph(12, 2 * 2, 4, rng)  # batch-major (b, h) graphs
+        return Problem(name, 2, 2, 64, group, group.copy(), 12, 12, row_ptr, cols, 19000,
+                       "tiny VSA-style, one graph per batch entry", graph_batches=2)
     raise KeyError(name)
 
 
@@ -284,8 +313,9 @@ def make_tensors(problem: Problem, names: Sequence[str] = ("q", "k", "v", "do"),
     for nm in names:
         slots = problem.kv_slots if nm in ("k", "v") else problem.q_slots
         grp = problem.kv_group if nm in ("k", "v") else problem.q_group
+        nh = problem.n_kv_heads if nm in ("k", "v") else problem.heads
         g = torch.Generator().manual_seed(problem.seed_base + seeds[nm])
-        t = torch.randn((b, problem.heads, slots, problem.head_dim), generator=g, dtype=torch.float32)
+        t = torch.randn((b, nh, slots, problem.head_dim), generator=g, dtype=torch.float32)
         t = t.to(torch.bfloat16)
         pad = torch.from_numpy(grp < 0)
         if bool(pad.any()):
