@@ -216,7 +216,8 @@ class Plan:
         return _entry_heads(self, which)
 
     def work(self, which: int) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
-        """(work [n, 32] int32, pages [e] int32, masks [e] uint64) of pass ``which`` (0 query-owned, 1 key-owned)."""
+        """(work [n, 32] int32, pages [e] int32, masks [e, 2] uint64) of pass ``which`` (0 query-owned, 1
+        key-owned); segment s of entry e is bits 16 (s % 4) of masks[e, s // 4]."""
         w = ctypes.POINTER(ctypes.c_int32)()
         p = ctypes.POINTER(ctypes.c_int32)()
         m = ctypes.POINTER(ctypes.c_uint64)()
@@ -225,7 +226,8 @@ class Plan:
                                        ctypes.byref(m), ctypes.byref(ne)), "spattn_plan_work")
         work = np.ctypeslib.as_array(w, shape=(nw.value * 32,)).reshape(-1, 32).copy() if nw.value else np.zeros((0, 32), np.int32)
         pages = np.ctypeslib.as_array(p, shape=(ne.value,)).copy() if ne.value else np.zeros(0, np.int32)
-        masks = np.ctypeslib.as_array(m, shape=(ne.value,)).copy() if ne.value else np.zeros(0, np.uint64)
+        masks = (np.ctypeslib.as_array(m, shape=(2 * ne.value,)).reshape(-1, 2).copy() if ne.value
+                 else np.zeros((0, 2), np.uint64))
         return work, pages, masks
 
 

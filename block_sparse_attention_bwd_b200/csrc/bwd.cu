@@ -397,7 +397,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
-    const int seg = code < 4 ? static_cast<int>(code) : -1;
+    const int seg = code < 8 ? static_cast<int>(code) : -1;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     bool ok = true;
     StepMasks<NP> raw;
@@ -704,7 +704,7 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
-    const int seg = code < 4 ? static_cast<int>(code) : -1;
+    const int seg = code < 8 ? static_cast<int>(code) : -1;
     const bool owned = code != 15u && row < 16 * wk.n_own;
     const int64_t slot = row < 16 * wk.n_own ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
     const bool loaded = row < 16 * wk.n_own && slot < q_slots;

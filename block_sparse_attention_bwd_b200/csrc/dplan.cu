@@ -13,7 +13,7 @@
 //     pages of every column group the graph lists for it (the column side's
 //     group -> page table), with the group's row mask on that page; sorts
 //     them by page in shared memory; merges them into one entry per page
-//     (four 16-bit segment masks); and compacts runs of pages whose attended
+//     (eight 16-bit segment masks); and compacts runs of pages whose attended
 //     rows share a 4-row group into strided entries, exactly as the host
 //     planner does;
 //   * the key-owned pass walks the transposed graph (key group -> query
@@ -43,7 +43,8 @@ __device__ __forceinline__ int dp_sub_group(uint32_t m) {
   return -1;
 }
 
-__device__ __forceinline__ uint32_t dp_fold(uint64_t m) {
+__device__ __forceinline__ uint32_t dp_fold(uint64_t lo, uint64_t hi) {
+  const uint64_t m = lo | hi;
   return static_cast<uint32_t>((m | (m >> 16) | (m >> 32) | (m >> 48)) & 0xFFFFu);
 }
 
@@ -137,8 +138,8 @@ __global__ void __launch_bounds__(1024) dp_scan_inclusive(int64_t* __restrict__ 
 struct ListArgs {
   // templates of this pass
   const int32_t* words;     // n_tmpl x 32
-  const int32_t* segs;      // n_tmpl x 4 (group id or -1)
-  const int32_t* seg_rows;  // n_tmpl x 4
+  const int32_t* segs;      // n_tmpl x kMaxSegments (group id or -1)
+  const int32_t* seg_rows;  // n_tmpl x kMaxSegments
   int64_t n_tmpl;
   // graph rows of the owned side's groups
   const int64_t* adj_ptr;
@@ -167,15 +168,16 @@ template <bool FILL>
 __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
   extern __shared__ uint8_t dp_smem[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(dp_smem);               // [kListCap]
-  int32_t* mpage = reinterpret_cast<int32_t*>(keys + kListCap);         // [kListCap]
+  uint64_t* mhi = keys + kListCap;                                      // [kListCap] segments 4..7
+  int32_t* mpage = reinterpret_cast<int32_t*>(mhi + kListCap);          // [kListCap]
   __shared__ int n_keys;
   const int64_t ti = blockIdx.x;
   const int32_t h = blockIdx.y;
   if (threadIdx.x == 0) n_keys = 0;
   __syncthreads();
   // gather (page << 20 | segment << 16 | row mask of the column group on the page)
-  for (int s = 0; s < 4; ++s) {
-    const int32_t g = a.segs[ti * 4 + s];
+  for (int s = 0; s < kMaxSegments; ++s) {
+    const int32_t g = a.segs[ti * kMaxSegments + s];
     if (g < 0) continue;
     int64_t r0, r1;
     dp_row(a.adj_ptr, static_cast<int64_t>(h) * a.n_src + g, a.adj_nnz, r0, r1, a.flag);
@@ -217,16 +219,19 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
     }
   }
   if (threadIdx.x != 0) return;
-  // merge: one entry per page, four 16-bit segment masks (in place: the
-  // merged index never passes the read index)
+  // merge: one entry per page, eight 16-bit segment masks in two words (in
+  // place: the merged index never passes the read index)
   int m = 0;
   for (int i = 0; i < n;) {
     const int32_t p = static_cast<int32_t>(keys[i] >> 20);
-    uint64_t mk = 0;
-    for (; i < n && static_cast<int32_t>(keys[i] >> 20) == p; ++i)
-      mk |= static_cast<uint64_t>(keys[i] & 0xFFFFu) << (16 * ((keys[i] >> 16) & 0xF));
+    uint64_t mk[2] = {0, 0};
+    for (; i < n && static_cast<int32_t>(keys[i] >> 20) == p; ++i) {
+      const int sg = static_cast<int>((keys[i] >> 16) & 0xF);
+      mk[sg >> 2] |= static_cast<uint64_t>(keys[i] & 0xFFFFu) << (16 * (sg & 3));
+    }
     mpage[m] = p;
-    keys[m] = mk;
+    keys[m] = mk[0];
+    mhi[m] = mk[1];
     ++m;
   }
   // strided compaction (the host planner's rule) and output
@@ -234,41 +239,45 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
   const int64_t off = FILL ? (slot == 0 ? 0 : a.counts[slot - 1]) : 0;
   int64_t cnt = 0;
   unsigned long long useful = 0;
-  const int32_t* sr = a.seg_rows + ti * 4;
-  auto emit = [&](int32_t ref, uint64_t mk) {
+  const int32_t* sr = a.seg_rows + ti * kMaxSegments;
+  auto emit = [&](int32_t ref, uint64_t lo, uint64_t hi) {
     if (FILL) {
       a.out_pages[off + cnt] = ref;
-      a.out_masks[off + cnt] = mk;
+      a.out_masks[2 * (off + cnt)] = lo;
+      a.out_masks[2 * (off + cnt) + 1] = hi;
     } else {
-      for (int s = 0; s < 4; ++s) useful += static_cast<unsigned long long>(sr[s]) * __popcll((mk >> (16 * s)) & 0xFFFFull);
+      for (int s = 0; s < kMaxSegments; ++s)
+        useful += static_cast<unsigned long long>(sr[s]) * __popcll(((s < 4 ? lo : hi) >> (16 * (s & 3))) & 0xFFFFull);
     }
     ++cnt;
   };
   for (int i = 0; i < m;) {
     const int32_t p = mpage[i];
-    const int k = a.strided ? dp_sub_group(dp_fold(keys[i])) : -1;
+    const int k = a.strided ? dp_sub_group(dp_fold(keys[i], mhi[i])) : -1;
     if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= a.col_slots) {
       int j = i;
       bool same = true;
       while (j < m && mpage[j] <= p + 3) {
-        if (dp_sub_group(dp_fold(keys[j])) != k) {
+        if (dp_sub_group(dp_fold(keys[j], mhi[j])) != k) {
           same = false;
           break;
         }
         ++j;
       }
       if (same && j - i >= 2) {
-        uint64_t mk = 0;
+        uint64_t mk[2] = {0, 0};
         for (int x = i; x < j; ++x) {
           const int jj = mpage[x] - p;
-          for (int sg = 0; sg < 4; ++sg) mk |= ((keys[x] >> (16 * sg + 4 * k)) & 0xFull) << (16 * sg + 4 * jj);
+          for (int sg = 0; sg < kMaxSegments; ++sg)
+            mk[sg >> 2] |= (((sg < 4 ? keys[x] : mhi[x]) >> (16 * (sg & 3) + 4 * k)) & 0xFull)
+                           << (16 * (sg & 3) + 4 * jj);
         }
-        emit(~static_cast<int32_t>(16 * p + 4 * k), mk);
+        emit(~static_cast<int32_t>(16 * p + 4 * k), mk[0], mk[1]);
         i = j;
         continue;
       }
     }
-    emit(p, keys[i]);
+    emit(p, keys[i], mhi[i]);
     ++i;
   }
   if (!FILL) {
@@ -362,8 +371,8 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     const int64_t nc = std::max<int64_t>(static_cast<int64_t>(H) * (d.tq.n + d.tk.n), 1);
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_counts), nc * sizeof(int64_t)));
     if (e != cudaSuccess) return SPATTN_ERR_OOM;
-    cudaFuncSetAttribute(dp_list<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 12);
-    cudaFuncSetAttribute(dp_list<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 12);
+    cudaFuncSetAttribute(dp_list<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 20);
+    cudaFuncSetAttribute(dp_list<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 20);
     d.ready = true;
   }
   // the plan keeps its own copy of the graph (inspection calls read it later)
@@ -407,7 +416,7 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     a.flag = flag;
     return a;
   };
-  const size_t smem = kListCap * 12;
+  const size_t smem = kListCap * 20;
   ListArgs la[2] = {args(true), args(false)};
   const PassTemplates* tt[2] = {&d.tq, &d.tk};
   WorkList* wls[2] = {&P->wq, &P->wk};
@@ -439,7 +448,7 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     const int64_t n_work = static_cast<int64_t>(P->batch) * H * tt[pass]->n;
     if (ensure(&wl.d_work, wl.cap_work, n_work * kWorkWords) != cudaSuccess ||
         ensure(&wl.d_pages, wl.cap_pages, total) != cudaSuccess ||
-        ensure(&wl.d_masks, wl.cap_masks, total) != cudaSuccess)
+        ensure(&wl.d_masks, wl.cap_masks, total * kMaskWords) != cudaSuccess)
       return SPATTN_ERR_OOM;
     la[pass].out_work = wl.d_work;
     la[pass].out_pages = wl.d_pages;

@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
-    const int seg = code < 4 ? static_cast<int>(code) : -1;
+    const int seg = code < 8 ? static_cast<int>(code) : -1;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;

@@ -33,7 +33,7 @@ struct TmaPages {
 struct TileArgs {
   const int32_t* work = nullptr;    // n_work x 32 words (see spattn_plan_work)
   const int32_t* pages = nullptr;   // column page ids
-  const uint64_t* masks = nullptr;  // 4 x 16-bit row masks per entry
+  const uint64_t* masks = nullptr;  // 8 x 16-bit row masks per entry (two words)
   int64_t n_work = 0;
   int64_t own_slots = 0;            // rows per (batch, head) of the owned side
   int64_t col_slots = 0;            // rows per (batch, head) of the column side

@@ -387,8 +387,9 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
             const int32_t b = adj.dst[e];
             for (int64_t x = col.gp_ptr[b]; x < col.gp_ptr[b + 1]; ++x) {
               const int64_t c = static_cast<int64_t>(j) * npc + col.gp_page[x];  // (head offset, page)
-              if (acc[c] == 0) touched.push_back(c);
-              acc[c] |= static_cast<uint64_t>(col.gp_mask[x]) << (16 * (s - s0));
+              if (acc[2 * c] == 0 && acc[2 * c + 1] == 0) touched.push_back(c);
+              const int sg = s - s0;
+              acc[2 * c + sg / 4] |= static_cast<uint64_t>(col.gp_mask[x]) << (16 * (sg % 4));
             }
           }
         }
@@ -402,7 +403,8 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       // attended rows (over all segments) lie in one 4-row group k, at least
       // two of them in the list, become one strided entry: the four groups
       // then cost one 16-column page instead of one page each.
-      auto fold = [](uint64_t m) {
+      auto fold = [&](int64_t c) {
+        const uint64_t m = acc[2 * c] | acc[2 * c + 1];
         return static_cast<uint32_t>((m | (m >> 16) | (m >> 32) | (m >> 48)) & 0xFFFFu);
       };
       size_t i = 0;
@@ -410,37 +412,40 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
         const int64_t c = touched[i];
         const int32_t p = static_cast<int32_t>(c % npc);
         const uint16_t jh = static_cast<uint16_t>(c / npc);
-        const int k = strided ? sub_group(fold(acc[c])) : -1;
+        const int k = strided ? sub_group(fold(c)) : -1;
         // (the bound keeps p + 3 inside the side, so c + 3 stays in head jh)
         if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= col.slots) {
           size_t j = i;
           bool same = true;
           while (j < touched.size() && touched[j] <= c + 3) {
-            if (sub_group(fold(acc[touched[j]])) != k) {
+            if (sub_group(fold(touched[j])) != k) {
               same = false;
               break;
             }
             ++j;
           }
           if (same && j - i >= 2) {
-            uint64_t m = 0;
+            uint64_t m[kMaskWords] = {0, 0};
             for (size_t x = i; x < j; ++x) {
               const int jj = static_cast<int>(touched[x] - c);
               for (int sg = 0; sg < kMaxSegments; ++sg)
-                m |= ((acc[touched[x]] >> (16 * sg + 4 * k)) & 0xFull) << (16 * sg + 4 * jj);
-              acc[touched[x]] = 0;
+                m[sg / 4] |= ((acc[2 * touched[x] + sg / 4] >> (16 * (sg % 4) + 4 * k)) & 0xFull)
+                             << (16 * (sg % 4) + 4 * jj);
+              acc[2 * touched[x]] = acc[2 * touched[x] + 1] = 0;
             }
             wl.pages.push_back(~static_cast<int32_t>(16 * p + 4 * k));
-            wl.masks.push_back(m);
+            wl.masks.push_back(m[0]);
+            wl.masks.push_back(m[1]);
             wl.heads.push_back(jh);
             i = j;
             continue;
           }
         }
         wl.pages.push_back(p);
-        wl.masks.push_back(acc[c]);
+        wl.masks.push_back(acc[2 * c]);
+        wl.masks.push_back(acc[2 * c + 1]);
         wl.heads.push_back(jh);
-        acc[c] = 0;
+        acc[2 * c] = acc[2 * c + 1] = 0;
         ++i;
       }
       const size_t n_entries = wl.pages.size() - static_cast<size_t>(w[2]);
@@ -490,7 +495,7 @@ void make_templates(const Side& own, PassTemplates& t) {
       std::memset(w, 0, sizeof(w));
       w[1] = npg;
       for (int i = 0; i < npg; ++i) w[4 + i] = tile[i];
-      int32_t rows[kMaxSegments] = {0, 0, 0, 0};
+      int32_t rows[kMaxSegments] = {};
       for (int r = 0; r < kTilePages * kPageRows; ++r) {
         uint32_t code = kCodeNotOwned;
         if (rg[r] == -1) {
@@ -499,7 +504,7 @@ void make_templates(const Side& own, PassTemplates& t) {
           for (int s = s0; s < s1; ++s)
             if (segs[s] == rg[r]) code = static_cast<uint32_t>(s - s0);
         }
-        if (code < 4) rows[code] += 1;
+        if (code < static_cast<uint32_t>(kMaxSegments)) rows[code] += 1;
         reinterpret_cast<uint32_t*>(w)[12 + r / 8] |= code << (4 * (r % 8));
       }
       t.words.insert(t.words.end(), w, w + kWorkWords);
@@ -567,7 +572,7 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
       std::vector<uint64_t> acc;
       for (int32_t u = t; u < n_units; u += n_threads) {
         const std::vector<int64_t> src = src_heads(u);
-        acc.assign(static_cast<size_t>(col.n_pages) * src.size(), 0);
+        acc.assign(static_cast<size_t>(col.n_pages) * src.size() * kMaskWords, 0);
         // Per unit, the packing with fewer physical pairs (then fewer items).
         if (mode != 2) build_head(own, col, adj, u, src, slot_tiles, part[u], acc, touched);
         if (mode != 1) {
@@ -610,7 +615,7 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   wl.heads.clear();
   wl.physical_pairs = 0;
   wl.pages.reserve(n_entries);
-  wl.masks.reserve(n_entries);
+  wl.masks.reserve(n_entries * kMaskWords);
   wl.heads.reserve(n_entries);
   for (auto& pt : part) {
     const int32_t off = static_cast<int32_t>(wl.pages.size());  // entry ranges are per part
@@ -764,7 +769,7 @@ int refresh_host(spattn_plan_s* P) {
   for (WorkList* w : {&P->wq, &P->wk}) {
     w->work.resize(static_cast<size_t>(w->n_work) * kWorkWords);
     w->pages.resize(static_cast<size_t>(w->n_entries_dev));
-    w->masks.resize(static_cast<size_t>(w->n_entries_dev));
+    w->masks.resize(static_cast<size_t>(w->n_entries_dev) * kMaskWords);
     if ((!w->work.empty() && cudaMemcpy(w->work.data(), w->d_work, w->work.size() * sizeof(int32_t),
                                         cudaMemcpyDeviceToHost) != cudaSuccess) ||
         (!w->pages.empty() && cudaMemcpy(w->pages.data(), w->d_pages, w->pages.size() * sizeof(int32_t),

@@ -15,7 +15,8 @@ namespace spattn {
 constexpr int kPageRows = 16;     // rows per page (the unit packed into tiles)
 constexpr int kBlockRows = 64;    // rows per logical Q block
 constexpr int kTilePages = 8;     // pages per 128-row tile
-constexpr int kMaxSegments = 4;   // distinct groups per work item (16-bit mask each)
+constexpr int kMaxSegments = 8;   // distinct groups per work item (16-bit mask each)
+constexpr int kMaskWords = 2;     // uint64 words per column entry: segment s at bits 16 (s % 4) of word s / 4
 constexpr int kWorkWords = 32;    // int32 words per work item
 
 // Page references (owned pages of a work item, column entries of its list):
@@ -59,7 +60,7 @@ struct Adjacency {
 struct WorkList {
   std::vector<int32_t> work;     // n_work * kWorkWords (all batches)
   std::vector<int32_t> pages;    // entries of one batch
-  std::vector<uint64_t> masks;
+  std::vector<uint64_t> masks;   // kMaskWords per entry
   // per entry: the query head of the entry within the item's K/V head group
   // (key-owned pass under grouped-query attention; 0 otherwise)
   std::vector<uint16_t> heads;
@@ -79,8 +80,8 @@ struct WorkList {
 // tiles of the layout split into items, without their column lists.
 struct PassTemplates {
   std::vector<int32_t> words;     // n x kWorkWords (bh and entry range set on the device)
-  std::vector<int32_t> segs;      // n x 4 group of each segment, -1 = none
-  std::vector<int32_t> seg_rows;  // n x 4 owned rows of each segment
+  std::vector<int32_t> segs;      // n x kMaxSegments group of each segment, -1 = none
+  std::vector<int32_t> seg_rows;  // n x kMaxSegments owned rows of each segment
   int64_t n = 0;
   int32_t* d_words = nullptr;
   int32_t* d_segs = nullptr;

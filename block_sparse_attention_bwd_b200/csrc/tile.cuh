@@ -46,8 +46,9 @@ __device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {
 }
 
 // The column-list masks of one step of NP pages for one row: each entry
-// holds 16 bits per segment, and a row reads only the 16-bit half-word of
-// its own segment.  `fetch` only issues the loads; the words are read by
+// holds 16 bits per segment in two 64-bit words (segment s at bits
+// 16 (s % 4) of word s / 4), and a row reads only the 16-bit half-word of its
+// own segment.  `fetch` only issues the loads; the words are read by
 // `bits`, an iteration later, so the load latency never stalls the row math
 // that runs in between.
 template <int NP>
@@ -55,11 +56,11 @@ struct StepMasks {
   uint32_t w[NP];
   // `seg` < 0 (a row without a segment) gives an all-zero mask.
   __device__ __forceinline__ void fetch(const uint64_t* __restrict__ masks, int first, int n, int seg) {
-    const uint16_t* h = reinterpret_cast<const uint16_t*>(masks + first) + (seg < 0 ? 0 : seg);
+    const uint16_t* h = reinterpret_cast<const uint16_t*>(masks + 2 * static_cast<int64_t>(first)) + (seg < 0 ? 0 : seg);
 #pragma unroll
     for (int j = 0; j < NP; ++j) {
       w[j] = 0u;
-      if (j < n && seg >= 0) w[j] = __ldg(h + 4 * j);
+      if (j < n && seg >= 0) w[j] = __ldg(h + 8 * j);
     }
   }
   // Row mask of the step: bit c of word c/32 <=> column c may be attended.

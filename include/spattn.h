@@ -244,11 +244,15 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
  *   [0] batch*heads + head of the owned side (query heads for which = 0,
  *       K/V heads for which = 1)   [1] owned page count n (<= 8)
  *   [2] first entry          [3] end entry (into pages/masks)
- *   [4..11] owned page ids   [12..27] 128 row codes, 4 bits each, row r in
- *   word 12 + r/8 at bit 4*(r%8): 0..3 = segment, 14 = owned row with no
- *   segment (padded), 15 = row not written by this item.
- * pages[e] is a page id of the other side; masks[e] holds four 16-bit row
- * masks over that page, one per segment (segment s in bits 16s..16s+15).
+ *   [4..11] owned page references   [12..27] 128 row codes, 4 bits each,
+ *   row r in word 12 + r/8 at bit 4*(r%8): 0..7 = segment, 14 = owned row
+ *   with no segment (padded), 15 = row not written by this item.
+ * A page reference p >= 0 is the page of slots 16p .. 16p+15; a negative
+ * value is a strided page with base slot b = ~value, whose row r is slot
+ * b + 16 (r / 4) + r % 4.  pages[e] is a page reference of the other side;
+ * masks[2e] and masks[2e+1] hold eight 16-bit row masks over that page, one
+ * per segment (segment s in bits 16 (s % 4) .. 16 (s % 4) + 15 of word
+ * masks[2e + s / 4]).
  * Entries are shared by all batch indices. */
 int spattn_plan_work(spattn_plan_t plan, int32_t which, const int32_t** work, int64_t* n_work,
                      const int32_t** pages, const uint64_t** masks, int64_t* n_entries);

@@ -25,7 +25,7 @@ def _items(plan, which):
     for w in work:
         n = int(w[1])
         key = (int(w[0]), tuple(int(x) for x in w[4:4 + n]), tuple(int(x) for x in w[12:28]))
-        lst = list(zip(pages[w[2]:w[3]].tolist(), masks[w[2]:w[3]].tolist()))
+        lst = list(zip(pages[w[2]:w[3]].tolist(), map(tuple, masks[w[2]:w[3]].tolist())))
         assert key not in out
         out[key] = lst
     return out

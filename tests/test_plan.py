@@ -77,10 +77,10 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
         if head_filter is not None and h not in head_filter:
             continue
         n_own, e0, e1 = int(w[1]), int(w[2]), int(w[3])
-        assert 1 <= n_own <= 8 and 0 <= e0 <= e1 <= pages.size
+        assert 1 <= n_own <= 8 and 0 <= e0 <= e1 <= pages.size and masks.shape == (pages.size, 2)
         codes = _codes(w)
         pg = pages[e0:e1].astype(np.int64)
-        mk = masks[e0:e1].astype(np.uint64)
+        mk = masks[e0:e1].astype(np.uint64)  # [entries, 2]
         first = np.array([pref_slots(x)[0] for x in pg], dtype=np.int64)
         assert np.all(np.diff(first) > 0), "column entries must be in ascending slot order"
         col_slot = np.stack([pref_slots(x) for x in pg]) if pg.size else np.zeros((0, 16), np.int64)
@@ -97,8 +97,8 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
             if c == 14:
                 assert own_group[slot] == -1
                 continue
-            assert c < 4 and own_group[slot] >= 0
-            bits = ((mk[:, None] >> (np.uint64(16 * c) + bits16)) & np.uint64(1)).astype(bool)
+            assert c < 8 and own_group[slot] >= 0
+            bits = ((mk[:, c // 4, None] >> (np.uint64(16 * (c % 4)) + bits16)) & np.uint64(1)).astype(bool)
             cols = col_slot[bits]
             assert np.all(cols < col_slots)
             for col in cols.tolist():
@@ -244,7 +244,7 @@ def _covered_heads(p, pl, which, batch):
                 continue
             slot = int(pref_slots(w[4 + r // 16])[r % 16])
             for e in range(e0, e1):
-                m = (int(masks[e]) >> (16 * c)) & 0xFFFF
+                m = (int(masks[e, c // 4]) >> (16 * (c % 4))) & 0xFFFF
                 if not m:
                     continue
                 cbh = bh if which == 0 else (bh // Hkv) * H + (bh % Hkv) * g + int(eh[e])
