@@ -7,14 +7,15 @@
 // (streaming) form used by FlashAttention-style kernels.
 //
 // One CTA runs one query-owned work item: up to 8 query pages (128 rows,
-// TMEM lanes) against its list of key pages, 8 pages (128 columns) per step.
+// TMEM lanes) against its list of key pages, 4 pages (64 columns) per step.
 //   warp 0      TMA producer: query pages once, then K and V pages of each
-//               step into an NS-deep ring, one 16-row box per page and
-//               64-column chunk (gathered straight from [B,H,S,D] memory);
+//               step into two-deep rings, one box per run of consecutive
+//               pages (or per strided page) and 64-column chunk, gathered
+//               straight from [B,H,S,D] memory;
 //   warp 1      allocates TMEM and issues tcgen05 MMAs from one thread:
 //               S_b = Q K^T into one of two TMEM buffers, then O += P V with
 //               P read from TMEM (bf16, written over S_b by the softmax);
-//   warps 4..7  one tile row per thread: exact mask from the step's page
+//   warps 2..5  one tile row per thread: exact mask from the step's page
 //               masks, running max with lazy rescaling, P in bf16 to TMEM,
 //               and the epilogue (O / l, LSE in natural log).
 // S is double-buffered, so the MMA of step c+1 overlaps the softmax of c.
@@ -74,7 +75,8 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   uint64_t* p_full = s_full + 2;    // [2]
   uint64_t* o_done = p_full + 2;
   uint64_t* drain = o_done + 1;
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* o_last = drain + 1;     // the last PV has finished
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(o_last + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
 
@@ -102,6 +104,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     }
     mbar_init(o_done, 1);
     mbar_init(drain, 1);
+    mbar_init(o_last, 1);
     fence_barrier_init();
   }
   if (warp == 1) tmem_alloc(tslot, 256);
@@ -195,7 +198,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       umma_commit_w(&k_empty[ks]);
       if (st >= 1 && !issue_pv(st - 1)) ok = false;
     }
-    if (ok && n_steps > 0) issue_pv(n_steps - 1);
+    if (ok && n_steps > 0 && issue_pv(n_steps - 1)) umma_commit_w(o_last);
     umma_commit_w(drain);
     mbar_wait_drain(drain, 0);
   } else {
@@ -280,23 +283,23 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
         f2_unpack(ls2[1], b0, b1);
         l += (a0 + a1) + (b0 + b1);
       }
-      if (st > 0) {
-        // Observe every PV completion in order (PV(st-1) here): a parity wait
-        // is only unambiguous while the barrier is at most one phase ahead.
+      if (st > 0 && __any_sync(0xffffffffu, resc)) {
+        // O must hold steps < st before this warp's rows are rescaled, so
+        // wait for PV(st-1) here (only here: P(st) needs no wait).  S(st) was
+        // issued after PV(st-2) finished and PV(st) waits for this step's
+        // arrival, so o_done has completed st-1 or st phases and the parity
+        // wait is unambiguous.
         ok = __all_sync(0xffffffffu, mbar_wait(o_done, (st - 1) & 1, ab));
         if (!ok) break;
-        if (__any_sync(0xffffffffu, resc)) {
-          // O holds steps < st: rescale this warp's rows before PV(st)
-          tc_fence_after();
+        tc_fence_after();
 #pragma unroll
-          for (int pc = 0; pc < D / 32; ++pc) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_off + pc * 32, r);
-            tmem_wait_ld();
+        for (int pc = 0; pc < D / 32; ++pc) {
+          uint32_t r[32];
+          tmem_ld32(tO + lane_off + pc * 32, r);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
-            tmem_st32(tO + lane_off + pc * 32, r);
-          }
+          for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha);
+          tmem_st32(tO + lane_off + pc * 32, r);
         }
       }
       tmem_wait_st();
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       mbar_arrive(&p_full[b]);
     }
     if (ok && n_steps > 0) {
-      ok = mbar_wait(o_done, (n_steps - 1) & 1, ab);
+      ok = mbar_wait(o_last, 0, ab);
       ok = __all_sync(0xffffffffu, ok);
       tc_fence_after();
     }
