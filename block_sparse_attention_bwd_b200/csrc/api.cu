@@ -138,6 +138,7 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
   a.col_slots = col_slots;
   a.scale = P->scale;
   a.err = P->d_err;
+  a.sched = P->d_sched;
   a.heads = P->heads;
   a.kv_heads = P->kv_heads;
   a.kv_group = P->heads / P->kv_heads;

@@ -133,18 +133,33 @@ constexpr int kAccWarp = 10;
 constexpr int kDkvThreads = 384;
 constexpr int kDoWarp = 11;
 
+// Persistent form: one CTA per SM takes work items from a device counter in
+// list order (longest first per head), so each SM keeps its rings and TMEM
+// across items.  Warp 0 fetches the next item and publishes it in a 4-deep
+// queue in shared memory; every other role reads the queue.  Stage, step and
+// item counters run across items, so every barrier keeps advancing one phase
+// at a time.  At an item boundary the producers load the next item's owned
+// K / V (once the last S^T / dP^T products of the previous item have read
+// them) and its first stages, and the first S^T / dP^T products of the next
+// item run while the row threads finish the previous item and write its dK /
+// dV; the accumulating products of the next item wait until those
+// accumulators have been read.
+constexpr int kItemQueue = 4;
+// readers of a queue slot: warps 1, 10, 11 and the 8 row-thread warps
+constexpr int kItemReaders = 11;
+
 template <int D>
 __global__ void __launch_bounds__(kDkvThreads, 1)
     dkdv_kernel(const __grid_constant__ TmaPages tm_k, const __grid_constant__ TmaPages tm_v,
                 const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_do,
-                const int32_t* __restrict__ work, const int32_t* __restrict__ col_pages,
-                const uint64_t* __restrict__ col_masks, const float* __restrict__ lse,
-                const float* __restrict__ delta, __nv_bfloat16* __restrict__ out_dk,
+                const int32_t* __restrict__ work, int64_t n_work, int* __restrict__ sched,
+                const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
+                const float* __restrict__ lse, const float* __restrict__ delta, __nv_bfloat16* __restrict__ out_dk,
                 __nv_bfloat16* __restrict__ out_dv, int64_t kv_slots, int64_t q_slots, float sl2, float scale,
                 int heads, int kv_heads, int kv_group, const uint16_t* __restrict__ col_heads, int* err) {
   using C = DkvCfg<D>;
   constexpr int QS = C::kQStages, DS = C::kDStages, NP = kBwdStepPages, SP = C::kStagePages;
-  constexpr int SPS = SP / NP;       // steps per stage
+  static_assert(SP == NP, "one MMA step per stage");
   constexpr int NH = SP * 16 / 32;  // stage columns per producer lane
   constexpr int kStageChunk = C::kStageChunk, kAugStage = C::kAugStage;
   extern __shared__ uint8_t smem_raw[];
@@ -157,29 +172,31 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   uint8_t* sDa = sQa + QS * kAugStage;               // -Delta slice of dO stage s at sDa + s*kAugStage
   uint8_t* sOnes = sDa + DS * kAugStage;             // ones slice of the owned K / V rows
   uint64_t* bars = reinterpret_cast<uint64_t*>(sOnes + kOnesBytes);
-  uint64_t* own_full = bars;
-  uint64_t* q_full = own_full + 1;
+  uint64_t* own_full = bars;          // the item's owned K / V rows have landed
+  uint64_t* own_free = own_full + 1;  // the item's last S^T / dP^T products have read them
+  uint64_t* q_full = own_free + 1;
   uint64_t* q_empty = q_full + QS;
   uint64_t* do_full = q_empty + QS;
   uint64_t* do_empty = do_full + DS;
   uint64_t* st_full = do_empty + DS;  // S^T, dP^T of a step are in the staging set
   uint64_t* st_free = st_full + 1;    // the row threads have loaded the staging set
   uint64_t* pt_full = st_free + 1;    // [2] P^T, dS^T of a step are in packed set p
-  uint64_t* acc_done = pt_full + 2;
-  uint64_t* acc_b = acc_done + 1;     // [2] dV, dK MMAs of the steps using packed set p finished
+  uint64_t* acc_done = pt_full + 2;   // the item's dV, dK products have finished
+  uint64_t* acc_free = acc_done + 1;  // the row threads have read the item's dV, dK
+  uint64_t* acc_b = acc_free + 1;     // [2] dV, dK MMAs of the steps using packed set p finished
   uint64_t* drain = acc_b + 2;        // [2] one per issuing warp
-  uint32_t* tslot = reinterpret_cast<uint32_t*>(drain + 2);
+  uint64_t* item_full = drain + 2;    // [kItemQueue]
+  uint64_t* item_empty = item_full + kItemQueue;  // [kItemQueue]
+  int32_t* items = reinterpret_cast<int32_t*>(item_empty + kItemQueue);  // [kItemQueue]
+  uint32_t* tslot = reinterpret_cast<uint32_t*>(items + kItemQueue);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tslot + 1);
   const Abort ab{abort_flag, err};
-
-  const Work wk = load_work(work, blockIdx.x);
-  const int n_cols = wk.e1 - wk.e0;
-  const int n_steps = (n_cols + NP - 1) / NP;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
     *abort_flag = 0;
     mbar_init(own_full, 1);
+    mbar_init(own_free, 1);
     mbar_init(&acc_b[0], 1);
     mbar_init(&acc_b[1], 1);
     mbar_init(&drain[1], 1);
@@ -195,7 +212,12 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     mbar_init(st_free, 256);
     for (int b = 0; b < 2; ++b) mbar_init(&pt_full[b], 256);
     mbar_init(acc_done, 1);
+    mbar_init(acc_free, 256);
     mbar_init(drain, 1);
+    for (int s = 0; s < kItemQueue; ++s) {
+      mbar_init(&item_full[s], 1);
+      mbar_init(&item_empty[s], kItemReaders);
+    }
     fence_barrier_init();
   }
   {
@@ -217,11 +239,23 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
   const uint32_t tmem = *tslot;
   const uint32_t tDV = tmem + 256, tDK = tmem + 256 + D;
 
+  // Item k of this CTA (k = 0, 1, ...): the readers wait for its queue slot,
+  // read it and release the slot; -1 ends the loop (also on abort).
+  auto read_item = [&](int k) -> int {
+    const int s = k % kItemQueue;
+    if (!__all_sync(0xffffffffu, mbar_wait(&item_full[s], (k / kItemQueue) & 1, ab))) return -1;
+    const int idx = *reinterpret_cast<volatile int32_t*>(&items[s]);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&item_empty[s]);
+    return idx;
+  };
+
   if (warp == 0 || warp == kDoWarp) {
     // ---------------- producers (whole warps): warp 0 = Q stages, warp 11 = dO stages ----------------
-    // Lane j < n owns page j of a step: it holds the page id (fetched one step
-    // ahead) and issues that page's TMA boxes; every lane also writes the
-    // augmented slice rows of two of the step's 64 query columns.
+    // Warp 0 also owns the item queue and loads each item's owned K / V rows.
+    // Lane j < n owns page j of a stage: it holds the page id (fetched one
+    // stage ahead) and issues that page's TMA boxes; every lane also writes
+    // the augmented slice rows of two of the stage's 64 query columns.
     const bool is_q = warp == 0;
     const int NS = is_q ? QS : DS;
     uint8_t* stage0 = is_q ? sQ : sDO;
@@ -230,99 +264,130 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     uint64_t* empty = is_q ? q_empty : do_empty;
     const TmaPages& tm = is_q ? tm_q : tm_do;
     const float* terms = is_q ? lse : delta;
-    if (is_q) {
-      if (lane == 0) {
-        tma_prefetch_desc(&tm_k.m64);
-        tma_prefetch_desc(&tm_v.m64);
-        mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
-      }
-      __syncwarp();
-      const int own_pid = lane < wk.n_own ? wk.own_page(lane) : 0;
-      load_page_runs<C::kNch>(sK, kChunkBytes, tm_k, own_pid, wk.n_own, wk.bh, own_full);
-      load_page_runs<C::kNch>(sV, kChunkBytes, tm_v, own_pid, wk.n_own, wk.bh, own_full);
-    }
+    const float inv_scale = 1.0f / scale;
     if (lane == 0) {
       tma_prefetch_desc(&tm.m64w);
       tma_prefetch_desc(&tm.m64);
-    }
-    // Lane j holds the page id of column page j of stages t and t+1, and the
-    // per-column term (LSE for Q, Delta for dO) of columns lane + 32h of
-    // stage t.  Both are fetched one stage ahead, and the fetched values are
-    // used only in the next iteration, so their global-load latency overlaps
-    // the waits and TMA issue of the current one instead of stalling it.
-    const float inv_scale = 1.0f / scale;
-    const int n_stages = (n_cols + SP - 1) / SP;
-    auto page_id = [&](int t) {
-      return (t < n_stages && lane < min(SP, n_cols - t * SP)) ? __ldg(col_pages + wk.e0 + t * SP + lane) : 0;
-    };
-    // Query head of a column page: the item's K/V head owns the query heads
-    // q_base .. q_base + kv_group - 1 (grouped-query attention); each entry
-    // names its offset.
-    const int q_base = (wk.bh / kv_heads) * heads + (wk.bh % kv_heads) * kv_group;
-    auto col_bh = [&](int t) {
-      return q_base + ((col_heads && t < n_stages && lane < min(SP, n_cols - t * SP))
-                           ? static_cast<int>(__ldg(col_heads + wk.e0 + t * SP + lane))
-                           : 0);
-    };
-    // Raw loads only (nothing here reads the loaded registers); a dead column
-    // (beyond the step or the tensor) loads a valid address and is zeroed
-    // where the value is used, through its bit in `live`.
-    auto fetch_terms = [&](int t, int pg_lane, int bh_lane, float (&x)[NH], uint32_t& live) {
-      const int n_t = min(SP, n_cols - t * SP);
-      live = 0u;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) {
-        const int idx = lane + 32 * h;  // column of the stage
-        const int pg = __shfl_sync(0xffffffffu, pg_lane, idx >> 4);
-        const int cb = __shfl_sync(0xffffffffu, bh_lane, idx >> 4);
-        const int64_t slot = pref_slot(pg, idx & 15);
-        const bool ok = t < n_stages && (idx >> 4) < n_t && slot < q_slots;
-        x[h] = __ldg(terms + static_cast<int64_t>(cb) * q_slots + (ok ? slot : 0));
-        live |= ok ? (1u << h) : 0u;
+      if (is_q) {
+        tma_prefetch_desc(&tm_k.m64);
+        tma_prefetch_desc(&tm_v.m64);
       }
-    };
-    // Augmented row of a column: -LSE / scale for Q (a column that attends
-    // nothing, LSE = -inf, is masked everywhere, like a dead one: zeros), or
-    // -Delta for dO.
-    auto term_row = [&](float t, bool ok) {
-      const float x = is_q ? t * inv_scale : t;
-      return aug_row(ok && isfinite(x) ? x : 0.f);
-    };
-    int pid = page_id(0), pid_next = page_id(1);
-    int cbh = col_bh(0), cbh_next = col_bh(1);
-    float xc[NH];
-    uint32_t livec;
-    fetch_terms(0, pid, cbh, xc, livec);
-    int issued = 0;
-    for (int t = 0; t < n_stages; ++t) {
-      const int s = t % NS;
-      const int n = min(SP, n_cols - t * SP);
-      const int pid_next2 = page_id(t + 2);
-      const int cbh_next2 = col_bh(t + 2);
-      float xn[NH];
-      uint32_t liven;
-      fetch_terms(t + 1, pid_next, cbh_next, xn, liven);
-      if (t >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((t / NS) - 1) & 1, ab))) break;
-#pragma unroll
-      for (int h = 0; h < NH; ++h)
-        *reinterpret_cast<uint4*>(aug0 + s * kAugStage + aug_row_off(lane + 32 * h)) = term_row(xc[h], (livec >> h) & 1u);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
-      __syncwarp();
-      load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, cbh, &full[s]);
-      issued = t + 1;
-      pid = pid_next;
-      pid_next = pid_next2;
-      cbh = cbh_next;
-      cbh_next = cbh_next2;
-      livec = liven;
-#pragma unroll
-      for (int h = 0; h < NH; ++h) xc[h] = xn[h];
     }
+    int T = 0;  // stages issued by this warp over all items
+    int own_loads = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      int idx;
+      if (is_q) {
+        const int s = k % kItemQueue;
+        if (k >= kItemQueue && !__all_sync(0xffffffffu, mbar_wait(&item_empty[s], ((k / kItemQueue) - 1) & 1, ab)))
+          break;
+        int v = 0;
+        if (lane == 0) {
+          v = atomicAdd(sched, 1);
+          v = v < n_work ? v : -1;
+          items[s] = v;
+          mbar_arrive(&item_full[s]);
+        }
+        idx = __shfl_sync(0xffffffffu, v, 0);
+      } else {
+        idx = read_item(k);
+      }
+      if (idx < 0) break;
+      const Work wk = load_work(work, idx);
+      const int n_cols = wk.e1 - wk.e0;
+      if (is_q) {
+        // owned K / V rows: their buffers are free once the previous item's
+        // last S^T / dP^T products have read them
+        if (k >= 1 && !__all_sync(0xffffffffu, mbar_wait(own_free, (k - 1) & 1, ab))) break;
+        if (lane == 0) mbar_arrive_expect_tx(own_full, 2 * wk.n_own * C::kNch * 2048);
+        __syncwarp();
+        const int own_pid = lane < wk.n_own ? wk.own_page(lane) : 0;
+        load_page_runs<C::kNch>(sK, kChunkBytes, tm_k, own_pid, wk.n_own, wk.bh, own_full);
+        load_page_runs<C::kNch>(sV, kChunkBytes, tm_v, own_pid, wk.n_own, wk.bh, own_full);
+        own_loads = k + 1;
+      }
+      // Lane j holds the page id of column page j of stages t and t+1, and the
+      // per-column term (LSE for Q, Delta for dO) of columns lane + 32h of
+      // stage t.  Both are fetched one stage ahead, and the fetched values are
+      // used only in the next iteration, so their global-load latency overlaps
+      // the waits and TMA issue of the current one instead of stalling it.
+      const int n_stages = (n_cols + SP - 1) / SP;
+      auto page_id = [&](int t) {
+        return (t < n_stages && lane < min(SP, n_cols - t * SP)) ? __ldg(col_pages + wk.e0 + t * SP + lane) : 0;
+      };
+      // Query head of a column page: the item's K/V head owns the query heads
+      // q_base .. q_base + kv_group - 1 (grouped-query attention); each entry
+      // names its offset.
+      const int q_base = (wk.bh / kv_heads) * heads + (wk.bh % kv_heads) * kv_group;
+      auto col_bh = [&](int t) {
+        return q_base + ((col_heads && t < n_stages && lane < min(SP, n_cols - t * SP))
+                             ? static_cast<int>(__ldg(col_heads + wk.e0 + t * SP + lane))
+                             : 0);
+      };
+      // Raw loads only (nothing here reads the loaded registers); a dead
+      // column (beyond the stage or the tensor) loads a valid address and is
+      // zeroed where the value is used, through its bit in `live`.
+      auto fetch_terms = [&](int t, int pg_lane, int bh_lane, float (&x)[NH], uint32_t& live) {
+        const int n_t = min(SP, n_cols - t * SP);
+        live = 0u;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) {
+          const int idx2 = lane + 32 * h;  // column of the stage
+          const int pg = __shfl_sync(0xffffffffu, pg_lane, idx2 >> 4);
+          const int cb = __shfl_sync(0xffffffffu, bh_lane, idx2 >> 4);
+          const int64_t slot = pref_slot(pg, idx2 & 15);
+          const bool okc = t < n_stages && (idx2 >> 4) < n_t && slot < q_slots;
+          x[h] = __ldg(terms + static_cast<int64_t>(cb) * q_slots + (okc ? slot : 0));
+          live |= okc ? (1u << h) : 0u;
+        }
+      };
+      // Augmented row of a column: -LSE / scale for Q (a column that attends
+      // nothing, LSE = -inf, is masked everywhere, like a dead one: zeros), or
+      // -Delta for dO.
+      auto term_row = [&](float t, bool okr) {
+        const float x = is_q ? t * inv_scale : t;
+        return aug_row(okr && isfinite(x) ? x : 0.f);
+      };
+      int pid = page_id(0), pid_next = page_id(1);
+      int cbh = col_bh(0), cbh_next = col_bh(1);
+      float xc[NH];
+      uint32_t livec;
+      fetch_terms(0, pid, cbh, xc, livec);
+      for (int t = 0; t < n_stages; ++t, ++T) {
+        const int s = T % NS;
+        const int n = min(SP, n_cols - t * SP);
+        const int pid_next2 = page_id(t + 2);
+        const int cbh_next2 = col_bh(t + 2);
+        float xn[NH];
+        uint32_t liven;
+        fetch_terms(t + 1, pid_next, cbh_next, xn, liven);
+        if (T >= NS && !__all_sync(0xffffffffu, mbar_wait(&empty[s], ((T / NS) - 1) & 1, ab))) {
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int h = 0; h < NH; ++h)
+          *reinterpret_cast<uint4*>(aug0 + s * kAugStage + aug_row_off(lane + 32 * h)) =
+              term_row(xc[h], (livec >> h) & 1u);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_expect_tx(&full[s], n * C::kNch * 2048);
+        __syncwarp();
+        load_page_runs<C::kNch>(stage0 + s * C::kStageTile, kStageChunk, tm, pid, n, cbh, &full[s]);
+        pid = pid_next;
+        pid_next = pid_next2;
+        cbh = cbh_next;
+        cbh_next = cbh_next2;
+        livec = liven;
+#pragma unroll
+        for (int h = 0; h < NH; ++h) xc[h] = xn[h];
+      }
+    }
+    // no copy may still be landing in shared memory when the CTA exits
     if (lane == 0) {
-      for (int t = max(0, issued - NS); t < issued; ++t) mbar_wait_drain(&full[t % NS], (t / NS) & 1);
-      if (is_q) mbar_wait_drain(own_full, 0);
+      for (int t = max(0, T - NS); t < T; ++t) mbar_wait_drain(&full[t % NS], (t / NS) & 1);
+      if (is_q && own_loads > 0) mbar_wait_drain(own_full, (own_loads - 1) & 1);
     }
   } else if (warp == 1) {
     // ---------------- S^T, dP^T issuer (warp-wide; one elected lane issues) ----------------
@@ -333,31 +398,42 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint64_t d_ones = sdesc_plain(smem_u32(sOnes), 128, 256);
     const uint64_t d_qa = sdesc_plain(smem_u32(sQa), 128, 256);
     const uint64_t d_da = sdesc_plain(smem_u32(sDa), 128, 256);
-    bool ok = __all_sync(0xffffffffu, mbar_wait(own_full, 0, ab));
-    tc_fence_after();
-    for (int st = 0; ok && st < n_steps; ++st) {
-      const int t = st / SPS, half = st % SPS, qs = t % QS, ds = t % DS;
-      const int n = min(NP, n_cols - st * NP);
-      const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      // the staging set is free once the row threads have loaded step st-1
-      bool w = (st < 1 || mbar_wait(st_free, (st - 1) & 1, ab)) && mbar_wait(&q_full[qs], (t / QS) & 1, ab);
-      if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+    int G = 0;  // steps over all items
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int idx = read_item(k);
+      if (idx < 0) break;
+      const Work wk = load_work(work, idx);
+      const int n_cols = wk.e1 - wk.e0;
+      const int n_steps = (n_cols + NP - 1) / NP;
+      ok = __all_sync(0xffffffffu, mbar_wait(own_full, k & 1, ab));
       tc_fence_after();
-      const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile + half * kHalfStage);
-      const uint64_t bd = sdesc_add(ddk, ds * C::kStageTile + half * kHalfStage);
+      for (int st = 0; ok && st < n_steps; ++st, ++G) {
+        const int qs = G % QS, ds = G % DS;
+        const int n = min(NP, n_cols - st * NP);
+        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+        // the staging set is free once the row threads have loaded step G-1
+        bool w = (G < 1 || mbar_wait(st_free, (G - 1) & 1, ab)) && mbar_wait(&q_full[qs], (G / QS) & 1, ab);
+        if (!__all_sync(0xffffffffu, w)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t bq = sdesc_add(dqk, qs * C::kStageTile);
+        const uint64_t bd = sdesc_add(ddk, ds * C::kStageTile);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
-                  sdesc_add(bq, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_ss_w(tmem, d_ones, sdesc_add(d_qa, qs * kAugStage + half * 2048), idesc_s, 1u);
-      if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (t / DS) & 1, ab))) { ok = false; break; }
-      tc_fence_after();
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss_w(tmem, sdesc_add(dk0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                    sdesc_add(bq, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+        umma_ss_w(tmem, d_ones, sdesc_add(d_qa, qs * kAugStage), idesc_s, 1u);
+        if (!__all_sync(0xffffffffu, mbar_wait(&do_full[ds], (G / DS) & 1, ab))) { ok = false; break; }
+        tc_fence_after();
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 64, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
-                  sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
-      umma_ss_w(tmem + 64, d_ones, sdesc_add(d_da, ds * kAugStage + half * 2048), idesc_s, 1u);
-      umma_commit_w(st_full);
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss_w(tmem + 64, sdesc_add(dv0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                    sdesc_add(bd, (kk >> 2) * kStageChunk + (kk & 3) * 32), idesc_s, kk > 0);
+        umma_ss_w(tmem + 64, d_ones, sdesc_add(d_da, ds * kAugStage), idesc_s, 1u);
+        umma_commit_w(st_full);
+      }
+      // the owned K / V buffers are free once these products have read them
+      umma_commit_w(own_free);
     }
     umma_commit_w(&drain[0]);
     mbar_wait_drain(&drain[0], 0);
@@ -366,28 +442,37 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const uint64_t dqm = sdesc_sw128(smem_u32(sQ), kStageChunk, 1024);    // Q stages, MN-major
     const uint64_t ddm = sdesc_sw128(smem_u32(sDO), kStageChunk, 1024);   // dO stages, MN-major
     const uint32_t idesc_acc = idesc_bf16(128, D, false, true);
+    int G = 0;
     bool ok = true;
-    for (int st = 0; ok && st < n_steps; ++st) {
-      const int b = st & 1, t = st / SPS, half = st % SPS, qs = t % QS, ds = t % DS;
-      // a stage is released after the MMAs of its last step
-      const bool stage_end = half == SPS - 1 || st + 1 == n_steps;
-      if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (st >> 1) & 1, ab))) { ok = false; break; }
+    for (int k = 0; ok; ++k) {
+      const int idx = read_item(k);
+      if (idx < 0) break;
+      const Work wk = load_work(work, idx);
+      const int n_cols = wk.e1 - wk.e0;
+      const int n_steps = (n_cols + NP - 1) / NP;
+      // the accumulators hold the previous item until its row threads read them
+      if (k >= 1 && !__all_sync(0xffffffffu, mbar_wait(acc_free, (k - 1) & 1, ab))) break;
       tc_fence_after();
-      const int n = min(NP, n_cols - st * NP);
-      const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile + half * kHalfStage);
-      const uint64_t bd = sdesc_add(ddm, ds * C::kStageTile + half * kHalfStage);
+      for (int st = 0; st < n_steps; ++st, ++G) {
+        const int b = G & 1, qs = G % QS, ds = G % DS;
+        if (!__all_sync(0xffffffffu, mbar_wait(&pt_full[b], (G >> 1) & 1, ab))) { ok = false; break; }
+        tc_fence_after();
+        const int n = min(NP, n_cols - st * NP);
+        const uint64_t bq = sdesc_add(dqm, qs * C::kStageTile);
+        const uint64_t bd = sdesc_add(ddm, ds * C::kStageTile);
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n) umma_ts_w(tDV, tmem + 128 + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      if (stage_end) umma_commit_w(&do_empty[ds]);
+        for (int j = 0; j < NP; ++j)
+          if (j < n) umma_ts_w(tDV, tmem + 128 + 64 * b + 8 * j, sdesc_add(bd, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+        umma_commit_w(&do_empty[ds]);
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n)
-          umma_ts_w(tDK, tmem + 160 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
-      if (stage_end) umma_commit_w(&q_empty[qs]);
-      umma_commit_w(&acc_b[b]);
+        for (int j = 0; j < NP; ++j)
+          if (j < n)
+            umma_ts_w(tDK, tmem + 160 + 64 * b + 8 * j, sdesc_add(bq, j * 2048), idesc_acc, (st > 0 || j > 0) ? 1u : 0u);
+        umma_commit_w(&q_empty[qs]);
+        umma_commit_w(&acc_b[b]);
+      }
+      if (ok) umma_commit_w(acc_done);  // every item, with or without steps
     }
-    if (ok && n_steps > 0) umma_commit_w(acc_done);
     umma_commit_w(&drain[1]);
     mbar_wait_drain(&drain[1], 0);
   } else {
@@ -396,107 +481,119 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t code = wk.row_code(row);
-    const int seg = code < 8 ? static_cast<int>(code) : -1;
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
+    int G = 0;
     bool ok = true;
-    StepMasks<NP> raw;
-    if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols), seg);
-    for (int st = 0; st < n_steps; ++st) {
-      const int b = st & 1;
-      const int N = 16 * min(NP, n_cols - st * NP);
-      const bool active = grp * 32 < N;
-      uint32_t mw[2];
-      raw.bits(mw);
-      // mask words of the next step load while this one computes
-      if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg);
-      ok = __all_sync(0xffffffffu, mbar_wait(st_full, st & 1, ab));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t a[32], d[32];
-      if (active) {
-        tmem_ld32(tmem + lane_off + grp * 32, a);
-        tmem_ld32(tmem + 64 + lane_off + grp * 32, d);
-        tmem_wait_ld();
-      }
-      tc_fence_before();
-      mbar_arrive(st_free);
-      // a = S^T - LSE/scale, d = dP^T - Delta (fp32, from the augmented MMAs)
-      uint32_t pp[16], pd[16];
-      if (active) {
-        const uint32_t m = grp ? mw[1] : mw[0];
-        if (m == 0xFFFFFFFFu) {
-          // every column allowed: no masking, all values finite
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1, s0, s1;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
-                      s1);
-            pp[i] = pack_bf16(p0, p1);
-            pd[i] = pack_bf16(s0, s1);
-          }
-        } else if (m == 0u) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            pp[i] = 0u;
-            pd[i] = 0u;
-          }
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1, s0, s1;
-            f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
-            float p0 = ex2(x0), p1 = ex2(x1);
-            if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
-            if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
-            f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
-                      s1);
-            pp[i] = pack_bf16(p0, p1);
-            // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
-            pd[i] = pack_bf16(p0 != 0.f ? s0 : 0.f, p1 != 0.f ? s1 : 0.f);
-          }
-        }
-      }
-      // Packed set b still feeds dV(st-2) / dK(st-2).  Every row thread waits,
-      // active or not, so that no arrival for step st can land in the
-      // pt_full phase of step st-2.
-      if (st >= 2 && !__all_sync(0xffffffffu, mbar_wait(&acc_b[b], ((st - 2) >> 1) & 1, ab))) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      if (active) {
-        tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 16, pp);
-        tmem_st16(tmem + 160 + 64 * b + lane_off + grp * 16, pd);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      mbar_arrive(&pt_full[b]);
-    }
-    if (ok && n_steps > 0) {
-      ok = __all_sync(0xffffffffu, mbar_wait(acc_done, 0, ab));
-      tc_fence_after();
-    }
-    if (ok) {
-      // group 0 writes dV, group 1 writes scale * dK
-      const bool owned = code != 15u && row < 16 * wk.n_own;
-      const int64_t slot = owned ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
-      const bool write = owned && slot < kv_slots;
-      const int64_t base = (static_cast<int64_t>(wk.bh) * kv_slots + slot) * D;
-      const uint32_t tacc = grp == 0 ? tDV : tDK;
-      __nv_bfloat16* out = grp == 0 ? out_dv : out_dk;
-      const float mul = grp == 0 ? 1.0f : scale;
-#pragma unroll
-      for (int pc = 0; pc < D / 32; ++pc) {
-        uint32_t r[32] = {};
-        if (n_steps > 0) {
-          tmem_ld32(tacc + lane_off + pc * 32, r);
+    for (int k = 0; ok; ++k) {
+      const int idx = read_item(k);
+      if (idx < 0) break;
+      const Work wk = load_work(work, idx);
+      const int n_cols = wk.e1 - wk.e0;
+      const int n_steps = (n_cols + NP - 1) / NP;
+      const uint32_t code = wk.row_code(row);
+      const int seg = code < 8 ? static_cast<int>(code) : -1;
+      StepMasks<NP> raw;
+      if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols), seg);
+      for (int st = 0; st < n_steps; ++st, ++G) {
+        const int b = G & 1;
+        const int N = 16 * min(NP, n_cols - st * NP);
+        const bool active = grp * 32 < N;
+        uint32_t mw[2];
+        raw.bits(mw);
+        // mask words of the next step load while this one computes
+        if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg);
+        ok = __all_sync(0xffffffffu, mbar_wait(st_full, G & 1, ab));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t a[32], d[32];
+        if (active) {
+          tmem_ld32(tmem + lane_off + grp * 32, a);
+          tmem_ld32(tmem + 64 + lane_off + grp * 32, d);
           tmem_wait_ld();
         }
-        if (write) store_row32(out + base + pc * 32, r, mul, n_steps == 0);
+        tc_fence_before();
+        mbar_arrive(st_free);
+        // a = S^T - LSE/scale, d = dP^T - Delta (fp32, from the augmented MMAs)
+        uint32_t pp[16], pd[16];
+        if (active) {
+          const uint32_t m = grp ? mw[1] : mw[0];
+          if (m == 0xFFFFFFFFu) {
+            // every column allowed: no masking, all values finite
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1, s0, s1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
+              const float p0 = ex2(x0), p1 = ex2(x1);
+              f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
+                        s1);
+              pp[i] = pack_bf16(p0, p1);
+              pd[i] = pack_bf16(s0, s1);
+            }
+          } else if (m == 0u) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              pp[i] = 0u;
+              pd[i] = 0u;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float x0, x1, s0, s1;
+              f2_unpack(f2_mul(f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1])), sl2x2), x0, x1);
+              float p0 = ex2(x0), p1 = ex2(x1);
+              if (!((m >> (2 * i)) & 1u)) p0 = 0.f;
+              if (!((m >> (2 * i + 1)) & 1u)) p1 = 0.f;
+              f2_unpack(f2_mul(f2_pack(p0, p1), f2_pack(__uint_as_float(d[2 * i]), __uint_as_float(d[2 * i + 1]))), s0,
+                        s1);
+              pp[i] = pack_bf16(p0, p1);
+              // masked entries: p = 0 exactly, so dS = 0 unless dP - Delta is not finite
+              pd[i] = pack_bf16(p0 != 0.f ? s0 : 0.f, p1 != 0.f ? s1 : 0.f);
+            }
+          }
+        }
+        // Packed set b still feeds dV(G-2) / dK(G-2).  Every row thread
+        // waits, active or not, so that no arrival for step G can land in
+        // the pt_full phase of step G-2.
+        if (G >= 2 && !__all_sync(0xffffffffu, mbar_wait(&acc_b[b], ((G - 2) >> 1) & 1, ab))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (active) {
+          tmem_st16(tmem + 128 + 64 * b + lane_off + grp * 16, pp);
+          tmem_st16(tmem + 160 + 64 * b + lane_off + grp * 16, pd);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(&pt_full[b]);
       }
+      if (!ok) break;
+      // acc_done completes once per item, after the item's last dV / dK products
+      ok = __all_sync(0xffffffffu, mbar_wait(acc_done, k & 1, ab));
+      if (!ok) break;
+      tc_fence_after();
+      {
+        // group 0 writes dV, group 1 writes scale * dK
+        const bool owned = code != 15u && row < 16 * wk.n_own;
+        const int64_t slot = owned ? pref_slot(wk.own_page(row >> 4), row & 15) : 0;
+        const bool write = owned && slot < kv_slots;
+        const int64_t base = (static_cast<int64_t>(wk.bh) * kv_slots + slot) * D;
+        const uint32_t tacc = grp == 0 ? tDV : tDK;
+        __nv_bfloat16* out = grp == 0 ? out_dv : out_dk;
+        const float mul = grp == 0 ? 1.0f : scale;
+#pragma unroll
+        for (int pc = 0; pc < D / 32; ++pc) {
+          uint32_t r[32] = {};
+          if (n_steps > 0) {
+            tmem_ld32(tacc + lane_off + pc * 32, r);
+            tmem_wait_ld();
+          }
+          if (write) store_row32(out + base + pc * 32, r, mul, n_steps == 0);
+        }
+      }
+      // the next item's dV / dK products may overwrite the accumulators
+      tc_fence_before();
+      mbar_arrive(acc_free);
     }
   }
 
@@ -860,9 +957,16 @@ static cudaError_t launch_dkdv_t(const TmaPages& tk, const TmaPages& tv, const T
   using C = DkvCfg<D>;
   cudaError_t e = cudaFuncSetAttribute(dkdv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess || a.n_work == 0) return e;
-  dkdv_kernel<D><<<static_cast<unsigned>(a.n_work), kDkvThreads, C::kSmem, st>>>(
-      tk, tv, tq, tdo, a.work, a.pages, a.masks, lse, delta, dk, dv, a.own_slots, a.col_slots, a.scale * kLog2e,
-      a.scale, a.heads, a.kv_heads, a.kv_group, a.col_heads, a.err);
+  // one persistent CTA per SM (at most one item each when there are fewer items)
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e == cudaSuccess) e = cudaMemsetAsync(a.sched, 0, sizeof(int), st);
+  if (e != cudaSuccess) return e;
+  const int64_t grid = std::min<int64_t>(a.n_work, std::max(sms, 1));
+  dkdv_kernel<D><<<static_cast<unsigned>(grid), kDkvThreads, C::kSmem, st>>>(
+      tk, tv, tq, tdo, a.work, a.n_work, a.sched, a.pages, a.masks, lse, delta, dk, dv, a.own_slots, a.col_slots,
+      a.scale * kLog2e, a.scale, a.heads, a.kv_heads, a.kv_group, a.col_heads, a.err);
   return cudaGetLastError();
 }
 

@@ -39,6 +39,7 @@ struct TileArgs {
   int64_t col_slots = 0;            // rows per (batch, head) of the column side
   float scale = 0.f;                // softmax scale
   int* err = nullptr;               // device error word
+  int* sched = nullptr;             // work-item counter of a persistent kernel (the launcher zeroes it)
   // Grouped-query attention: query head h reads K/V head h / kv_group
   // (heads = query heads, kv_heads = heads / kv_group).  For the key-owned
   // pass, entry e's column head is the item's first query head + col_heads[e].

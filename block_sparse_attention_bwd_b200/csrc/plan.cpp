@@ -752,6 +752,7 @@ void free_plan_device(spattn_plan_s* P) {
   cudaFree(P->d_q_fill);
   cudaFree(P->d_k_fill);
   cudaFree(P->d_err);
+  cudaFree(P->d_sched);
   cudaFree(P->d_delta);
   for (auto& e : P->events) {
     cudaEventDestroy(e.start);
@@ -882,6 +883,7 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if ((st = upload(P->q_fill, &P->d_q_fill, bytes))) return st;
   if ((st = upload(P->k_fill, &P->d_k_fill, bytes))) return st;
   if (cudaMalloc(reinterpret_cast<void**>(&P->d_err), sizeof(int)) != cudaSuccess) return SPATTN_ERR_OOM;
+  if (cudaMalloc(reinterpret_cast<void**>(&P->d_sched), sizeof(int)) != cudaSuccess) return SPATTN_ERR_OOM;
   if (cudaMemset(P->d_err, 0, sizeof(int)) != cudaSuccess) return SPATTN_ERR_CUDA;
   const size_t delta_bytes = static_cast<size_t>(L->batch) * L->heads * L->q_slots * sizeof(float);
   if (cudaMalloc(reinterpret_cast<void**>(&P->d_delta), delta_bytes) != cudaSuccess) return SPATTN_ERR_OOM;

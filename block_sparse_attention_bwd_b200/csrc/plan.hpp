@@ -132,6 +132,7 @@ struct spattn_plan_s {
   int32_t* d_q_fill = nullptr;
   int32_t* d_k_fill = nullptr;
   int* d_err = nullptr;        // device error word
+  int* d_sched = nullptr;      // work-item counter of the persistent dK/dV kernel
   float* d_delta = nullptr;    // [batch, heads, q_slots] rowsum(dO * O)
   spattn::DevPlanner dp;        // device planner state
   bool host_stale = false;      // the work lists / graph were rebuilt on the device
