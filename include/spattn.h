@@ -169,7 +169,9 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
                void* stream);
 
 /* Backward: dQ, dK, dV given O and LSE from spattn_fwd and the loss
- * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O).
+ * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O) and the
+ * plan's work-item counter of the persistent dK/dV kernel, so backward calls
+ * on one plan must be ordered (one stream, or events between streams).
  * dK and dV are accumulated per owned key tile and written once, with no
  * atomics: the KPage abstract (zhuanzhiai.com paper page) keeps the graph
  * exact in the backward pass by letting the K/V side own its pages.  The
