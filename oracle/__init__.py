@@ -14,7 +14,9 @@ gradients, which is what this package computes, in float64, with NumPy.
 Every function here is pinned by ``tests/test_oracle.py`` against something
 other than itself (dense attention from ``torch`` on a full graph, closed
 forms for single-key rows and zero queries, central finite differences,
-brute-force counts).
+brute-force counts).  ``oracle.fp8`` (the E4M3 codec and per-slice quantiser
+of the FP8 forward) is pinned by ``tests/test_oracle_fp8.py`` against
+hand-computed codes of the format and a brute-force nearest-value search.
 """
 
 from .attention import (  # noqa: F401
@@ -34,3 +36,4 @@ from .plan import (  # noqa: F401
     useful_pairs_closed_form,
     bsa_physical_pairs,
 )
+from . import fp8  # noqa: F401,E402
