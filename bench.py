@@ -329,6 +329,50 @@ def device_plan_ms(plan, p, dev, reps=5):
     return statistics.median(times)
 
 
+def measure_fwd_fp8(plan, x, out, U, D, steps, peak_burst, flush, scratch):
+    """The FP8 forward on the same plan and inputs: Q and K quantised once
+    to E4M3 (timed on its own), then `steps` timed spattn_fwd_fp8 calls
+    (CUDA events on the launch stream, L2 flushed between calls when the
+    inputs fit in it).  Reported against the mixed peak of its two products:
+    S at the fp8 rate (2x the measured bf16 burst, the nominal ratio) and
+    P V at the bf16 rate."""
+    import torch
+
+    import block_sparse_attention_bwd_b200 as sp
+
+    stream = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for _ in range(2):
+        q8, qds = sp.quantize_fp8(x["q"])
+        k8, kds = sp.quantize_fp8(x["k"])
+    torch.cuda.synchronize()
+    e0.record(stream)
+    q8, qds = sp.quantize_fp8(x["q"])
+    k8, kds = sp.quantize_fp8(x["k"])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    quant_ms = e0.elapsed_time(e1)
+    for _ in range(3):
+        sp.spattn_fwd_fp8(q8, k8, qds, kds, x["v"], plan, o=out["o"], lse=out["lse"])
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        if flush:
+            scratch.zero_()
+        a.record(stream)
+        sp.spattn_fwd_fp8(q8, k8, qds, kds, x["v"], plan, o=out["o"], lse=out["lse"])
+        b.record(stream)
+    torch.cuda.synchronize()
+    sp.spattn_check(plan)
+    t = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    tflops = 4 * D * U / (t / 1e3) / 1e12
+    peak_mixed = 2.0 / (1.0 / (2.0 * peak_burst) + 1.0 / peak_burst)
+    return {"value": tflops, "unit": "TFLOP/s", "ms_per_step": t, "steps": steps, "quantize_q_k_ms": quant_ms,
+            "dtype": "e4m3 Q, K (S = Q K^T on kind::f8f6f4); bf16 P, V, O",
+            "peak_mixed": peak_mixed, "frac_of_mixed_peak": tflops / peak_mixed,
+            "pct_of_bf16_peak": 100 * tflops / peak_burst}
+
+
 def measure_workload(name, steps, warmup, dev, peak_burst):
     """fwd and fwd+bwd useful-pair TFLOP/s of one workload on resident inputs
     (CUDA events on the launch stream, L2 flushed between steps when the
@@ -570,6 +614,10 @@ def run_ours(args):
                           f"extrapolated linearly by useful pairs to the whole workload"),
                "fwd_value": 4 * D * U / tf / 1e12}
 
+    fp8 = None
+    if rank == 0 and world == 1 and D == 128 and args.fp8_steps > 0:
+        fp8 = measure_fwd_fp8(plan, x, out, U, D, args.fp8_steps, peak_burst, flush, scratch)
+
     dplan_ms = device_plan_ms(plan, p, dev) if rank == 0 else None
 
     # ---------------- every other large workload, measured the same way ----------------
@@ -594,6 +642,7 @@ def run_ours(args):
         "fwd": {"value": fwd_tflops, "unit": "TFLOP/s", "ms_per_step": t_fwd / K * 1e3,
                 "pct_of_bf16_peak": 100 * fwd_tflops / world / peak_burst},
         "bwd_ms_per_step": t_bwd / K * 1e3,
+        "fwd_fp8": fp8,
         "fwd_bwd_14D_value": 14 * D * U * world * K / t_total / 1e12,
         "pct_of_bf16_peak": 100 * value / world / peak_burst,
         "pairs": {"useful": U, "physical_fwd": st["physical_pairs_fwd"], "physical_dkdv": st["physical_pairs_dkdv"],
@@ -628,6 +677,8 @@ def main():
     ap.add_argument("--other-workloads", default="vsa,svg2,full",
                     help="after the headline, measure these workloads too (comma list; empty = none)")
     ap.add_argument("--other-steps", type=int, default=8)
+    ap.add_argument("--fp8-steps", type=int, default=10,
+                    help="timed calls of the FP8 (E4M3 Q/K) forward on the same workload; 0 skips it")
     ap.add_argument("--heads", type=int, default=0,
                     help="profile a slice: keep the layout, use the graph of the first N heads only")
     args = ap.parse_args()

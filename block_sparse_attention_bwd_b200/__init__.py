@@ -39,6 +39,7 @@ ENTRY_POINTS = (
     "spattn_plan", "spattn_fwd", "spattn_bwd", "spattn_bwd_noalloc", "spattn_check", "spattn_plan_stats", "spattn_profile",
     "spattn_profile_read", "spattn_plan_pages", "spattn_plan_qblocks", "spattn_plan_work", "spattn_plan_destroy",
     "spattn_status_string", "spattn_wait_selftest", "spattn_plan_set_graph_device", "spattn_plan_entry_heads",
+    "spattn_quantize_fp8", "spattn_fwd_fp8",
 )
 
 
@@ -90,6 +91,8 @@ def _lib():
         lib.spattn_plan.argtypes = [ctypes.POINTER(_Layout), ctypes.POINTER(_Graph), ctypes.POINTER(P)]
         lib.spattn_fwd.argtypes = [P, P, P, P, P, P, P]
         lib.spattn_bwd.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
+        lib.spattn_quantize_fp8.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
+        lib.spattn_fwd_fp8.argtypes = [P, P, P, P, P, P, P, P, P]
         lib.spattn_bwd_noalloc.argtypes = [P, P, P, P, P, P, P, P, P, P, P]
         lib.spattn_check.argtypes = [P, P]
         lib.spattn_wait_selftest.argtypes = [P, I64, P]
@@ -275,6 +278,43 @@ def spattn_fwd(q, k, v, plan: Plan, o=None, lse=None, stream=None):
     _need(lse, "lse", qs[:3], torch.float32)
     _check(_lib().spattn_fwd(_ptr(q), _ptr(k), _ptr(v), plan.handle, _ptr(o), _ptr(lse), _stream_handle(stream)),
            "spattn_fwd")
+    return o, lse
+
+
+def quantize_fp8(x, stream=None):
+    """E4M3 codes (uint8, same shape) and per-(batch, head) descale factors
+    (float32 [B, H]) of a bf16 tensor [B, H, S, D], one slice per (batch, head)."""
+    import torch
+
+    if x.dim() != 4 or x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous():
+        raise ValueError("quantize_fp8: x must be a contiguous CUDA bf16 tensor [B, H, S, D]")
+    B, H, S, D = x.shape
+    x8 = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    descale = torch.empty((B, H), dtype=torch.float32, device=x.device)
+    _check(_lib().spattn_quantize_fp8(_ptr(x), B * H, S, D, _ptr(x8), _ptr(descale), _stream_handle(stream)),
+           "spattn_quantize_fp8")
+    return x8, descale
+
+
+def spattn_fwd_fp8(q8, k8, q_descale, k_descale, v, plan: Plan, o=None, lse=None, stream=None):
+    """O and LSE of attention over the dequantised E4M3 Q and K (see quantize_fp8)."""
+    import torch
+
+    qs = (plan.batch, plan.heads, plan.q_slots, plan.head_dim)
+    ks = (plan.batch, plan.kv_heads, plan.kv_slots, plan.head_dim)
+    _need(q8, "q8", qs, torch.uint8)
+    _need(k8, "k8", ks, torch.uint8)
+    _need(v, "v", ks, torch.bfloat16)
+    _need(q_descale, "q_descale", qs[:2], torch.float32)
+    _need(k_descale, "k_descale", ks[:2], torch.float32)
+    if o is None:
+        o = torch.empty(qs, dtype=torch.bfloat16, device=q8.device)
+    if lse is None:
+        lse = torch.empty(qs[:3], dtype=torch.float32, device=q8.device)
+    _need(o, "o", qs, torch.bfloat16)
+    _need(lse, "lse", qs[:3], torch.float32)
+    _check(_lib().spattn_fwd_fp8(_ptr(q8), _ptr(k8), _ptr(q_descale), _ptr(k_descale), _ptr(v), plan.handle, _ptr(o),
+                                 _ptr(lse), _stream_handle(stream)), "spattn_fwd_fp8")
     return o, lse
 
 

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libspattn.so")
-SOURCES = ["plan.cpp", "api.cu", "fwd.cu", "bwd.cu", "noalloc.cu", "selftest.cu", "dplan.cu"]
+SOURCES = ["plan.cpp", "api.cu", "fwd.cu", "bwd.cu", "noalloc.cu", "selftest.cu", "dplan.cu", "quant.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC,-O3,-pthread", "-I" + os.path.join(ROOT, "include")]
 

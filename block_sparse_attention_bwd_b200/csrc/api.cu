@@ -35,18 +35,23 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [rows_per_bh, head_dim] bf16 matrices stacked over batch*heads; boxes of
-// `box_rows` rows x 64 columns, 128-byte swizzle (the layout the MMA
-// descriptors expect).  Rows past the end of a (batch, head) read as zeros.
-bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows) {
+// Element types of the mapped tensors: bf16, or one-byte E4M3 codes (moved
+// as bytes).  Every box row is 128 bytes (64 bf16 or 128 codes), the width of
+// the 128-byte swizzle the MMA descriptors expect.
+CUtensorMapDataType map_type(int eb) { return eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16; }
+
+// [rows_per_bh, head_dim] matrices stacked over batch*heads; boxes of
+// `box_rows` rows x one 128-byte chunk, 128-byte swizzle.  Rows past the end
+// of a (batch, head) read as zeros.
+bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows, int eb = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(bh)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * 2, static_cast<cuuint64_t>(head_dim) * 2 * rows};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(head_dim) * eb, static_cast<cuuint64_t>(head_dim) * eb * rows};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t es[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, es,
+  return fn(m, map_type(eb), 3, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -55,15 +60,18 @@ bool make_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64
 // every chunk of those rows, chunk after chunk.  The chunk stride (128 B) is
 // below the row stride; a tiled map only needs each stride to be a multiple
 // of 16 bytes.
-bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows) {
+bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int box_rows,
+                   int eb = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const int nch = head_dim / 64;
-  cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nch), static_cast<cuuint64_t>(bh)};
-  cuuint64_t strides[3] = {static_cast<cuuint64_t>(head_dim) * 2, 128, static_cast<cuuint64_t>(head_dim) * 2 * rows};
-  cuuint32_t box[4] = {64, static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(nch), 1};
+  const int nch = head_dim * eb / 128;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(head_dim) * eb;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(128 / eb), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(nch),
+                        static_cast<cuuint64_t>(bh)};
+  cuuint64_t strides[3] = {row_bytes, 128, row_bytes * rows};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(128 / eb), static_cast<cuuint32_t>(box_rows), static_cast<cuuint32_t>(nch), 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+  return fn(m, map_type(eb), 4, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -73,31 +81,31 @@ bool make_wide_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, 
 // dimension; every box the kernels request lies inside one (batch, head),
 // because the planner only forms a strided page when all 16 of its slots
 // exist.
-bool make_strided_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
+bool make_strided_map(CUtensorMap* m, const void* ptr, int head_dim, int64_t rows, int64_t bh, int eb = 2) {
   auto fn = encode_fn();
   if (!fn) return false;
-  const cuuint64_t row_bytes = static_cast<cuuint64_t>(head_dim) * 2;
+  const cuuint64_t row_bytes = static_cast<cuuint64_t>(head_dim) * eb;
   cuuint64_t dims[5] = {static_cast<cuuint64_t>(head_dim), 4, 4, static_cast<cuuint64_t>(rows),
                         static_cast<cuuint64_t>(bh)};
   cuuint64_t strides[4] = {row_bytes, 16 * row_bytes, row_bytes, row_bytes * static_cast<cuuint64_t>(rows)};
-  cuuint32_t box[5] = {64, 4, 4, 1, 1};
+  cuuint32_t box[5] = {static_cast<cuuint32_t>(128 / eb), 4, 4, 1, 1};
   cuuint32_t es[5] = {1, 1, 1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides, box, es,
+  return fn(m, map_type(eb), 5, const_cast<void*>(ptr), dims, strides, box, es,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool make_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh) {
-  if (!make_strided_map(&t->m4s, ptr, head_dim, rows, bh)) return false;
-  if (!make_map(&t->m16, ptr, head_dim, rows, bh, 16) || !make_map(&t->m32, ptr, head_dim, rows, bh, 32) ||
-      !make_map(&t->m64, ptr, head_dim, rows, bh, 64))
+bool make_pages(TmaPages* t, const void* ptr, int head_dim, int64_t rows, int64_t bh, int eb = 2) {
+  if (!make_strided_map(&t->m4s, ptr, head_dim, rows, bh, eb)) return false;
+  if (!make_map(&t->m16, ptr, head_dim, rows, bh, 16, eb) || !make_map(&t->m32, ptr, head_dim, rows, bh, 32, eb) ||
+      !make_map(&t->m64, ptr, head_dim, rows, bh, 64, eb))
     return false;
-  if (!make_wide_map(&t->m128w, ptr, head_dim, rows, bh, 128)) return false;
-  if (head_dim == 64) {
+  if (!make_wide_map(&t->m128w, ptr, head_dim, rows, bh, 128, eb)) return false;
+  if (head_dim * eb == 128) {  // one chunk per row
     t->m64w = t->m64;
     return true;
   }
-  return make_wide_map(&t->m64w, ptr, head_dim, rows, bh, 64);
+  return make_wide_map(&t->m64w, ptr, head_dim, rows, bh, 64, eb);
 }
 
 bool aligned16(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -208,6 +216,47 @@ int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, 
   auto* O = static_cast<__nv_bfloat16*>(o);
   cudaError_t e = timed(plan, SPATTN_K_FWD, s, [&] {
     return launch_fwd(D, tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), O, lse, s);
+  });
+  if (e == cudaSuccess && !plan->q_fill.empty())
+    e = timed(plan, SPATTN_K_FILL, s, [&] {
+      return launch_fill(D, plan->d_q_fill, static_cast<int64_t>(plan->q_fill.size() / 2), bh, plan->q.slots, O,
+                         nullptr, lse, s);
+    });
+  return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
+}
+
+int spattn_quantize_fp8(const void* x, int64_t bh, int64_t rows, int head_dim, void* x8, float* descale,
+                        void* stream) {
+  if (bh < 0 || rows < 0 || (head_dim != 64 && head_dim != 128)) return SPATTN_ERR_INVALID_ARG;
+  if (bh == 0) return SPATTN_OK;
+  if (!aligned16(x) || !aligned16(x8) || !descale || (reinterpret_cast<uintptr_t>(descale) & 3u))
+    return SPATTN_ERR_INVALID_ARG;
+  const cudaError_t e = launch_quantize_e4m3(static_cast<const __nv_bfloat16*>(x), bh, rows * head_dim,
+                                             static_cast<uint8_t*>(x8), descale, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? SPATTN_OK : SPATTN_ERR_CUDA;
+}
+
+int spattn_fwd_fp8(const void* q8, const void* k8, const float* q_descale, const float* k_descale, const void* v,
+                   spattn_plan_t plan, void* o, float* lse, void* stream) {
+  if (!plan) return SPATTN_ERR_INVALID_ARG;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o) || !aligned16(lse) || !q_descale ||
+      !k_descale || (reinterpret_cast<uintptr_t>(q_descale) & 3u) || (reinterpret_cast<uintptr_t>(k_descale) & 3u))
+    return SPATTN_ERR_INVALID_ARG;
+  const int D = plan->head_dim;
+  if (D != 128) return SPATTN_ERR_UNSUPPORTED;
+  const int64_t bh = static_cast<int64_t>(plan->batch) * plan->heads;
+  const int64_t bh_kv = static_cast<int64_t>(plan->batch) * plan->kv_heads;
+  TmaPages tq, tk, tv;
+  if (!make_pages(&tq, q8, D, plan->q.slots, bh, 1) || !make_pages(&tk, k8, D, plan->k.slots, bh_kv, 1) ||
+      !make_pages(&tv, v, D, plan->k.slots, bh_kv))
+    return SPATTN_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  auto* O = static_cast<__nv_bfloat16*>(o);
+  cudaError_t e = timed(plan, SPATTN_K_FWD, s, [&] {
+    return launch_fwd_e4m3(tq, tk, tv, tile_args(plan, plan->wq, plan->q.slots, plan->k.slots), q_descale, k_descale,
+                           O, lse, s);
   });
   if (e == cudaSuccess && !plan->q_fill.empty())
     e = timed(plan, SPATTN_K_FILL, s, [&] {

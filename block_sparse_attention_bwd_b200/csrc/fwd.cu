@@ -33,14 +33,20 @@ using namespace dev;
 constexpr int kFwdStepPages = 4;
 constexpr int kFwdStageChunk = 64 * 128;  // one 64-column chunk of a 64-row stage
 
-template <int D>
+// F8: Q and K are E4M3 codes (one byte per element, so a 128-byte swizzle
+// row holds 128 of them) and S = Q K^T is a kind::f8f6f4 product; V, P and O
+// stay bf16.
+template <int D, bool F8>
 struct FwdCfg {
-  static constexpr int kNch = D / 64;                     // 64-column chunks
-  static constexpr int kTile = kNch * kChunkBytes;        // 128-row query tile
-  static constexpr int kStage = kNch * kFwdStageChunk;    // 64-row K or V stage
-  static constexpr int kKStages = (D == 128) ? 2 : 4;     // K ring depth
-  static constexpr int kVStages = (D == 128) ? 2 : 4;     // V ring depth
-  static constexpr int kSmem = kTile + (kKStages + kVStages) * kStage + 1024 + 512;
+  static constexpr int kNch = D / 64;                       // 64-column bf16 chunks (V)
+  static constexpr int kQKNch = F8 ? D / 128 : D / 64;      // 128-byte chunks of a Q or K row
+  static constexpr int kTile = kQKNch * kChunkBytes;        // 128-row query tile
+  static constexpr int kKStage = kQKNch * kFwdStageChunk;   // 64-row K stage
+  static constexpr int kVStage = kNch * kFwdStageChunk;     // 64-row V stage
+  static constexpr int kKStages = (D == 128 && !F8) ? 2 : 4;  // K ring depth
+  static constexpr int kVStages = (D == 128) ? 2 : 4;         // V ring depth
+  static constexpr int kSmem = kTile + kKStages * kKStage + kVStages * kVStage + 1024 + 512;
+  static_assert(!F8 || D == 128, "the E4M3 forward has D = 128 (one 128-byte row per chunk)");
 };
 
 // Rescale O only when the running max grows by more than 2^8 (log2 units):
@@ -51,21 +57,22 @@ constexpr float kRescaleThreshold = 8.0f;
 // threads (warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31).
 constexpr int kFwdThreads = 192;
 
-template <int D>
+template <int D, bool F8>
 __global__ void __launch_bounds__(kFwdThreads, 2)
     fwd_kernel(const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_k,
                const __grid_constant__ TmaPages tm_v, const int32_t* __restrict__ work,
                const int32_t* __restrict__ col_pages, const uint64_t* __restrict__ col_masks,
                __nv_bfloat16* __restrict__ out_o, float* __restrict__ out_lse, int64_t q_slots, float sl2,
-               int heads, int kv_group, int* err) {
-  using C = FwdCfg<D>;
+               int heads, int kv_group, const float* __restrict__ q_descale, const float* __restrict__ k_descale,
+               int* err) {
+  using C = FwdCfg<D, F8>;
   constexpr int KS = C::kKStages, VS = C::kVStages, NP = kFwdStepPages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* sQ = smem;
-  uint8_t* sK = smem + C::kTile;          // K stage s at sK + s*kStage
-  uint8_t* sV = sK + KS * C::kStage;      // V stage s at sV + s*kStage
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kStage);
+  uint8_t* sK = smem + C::kTile;          // K stage s at sK + s*kKStage
+  uint8_t* sV = sK + KS * C::kKStage;     // V stage s at sV + s*kVStage
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + VS * C::kVStage);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;
   uint64_t* k_empty = k_full + KS;
@@ -124,10 +131,11 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       tma_prefetch_desc(&tm_v.m64);
       tma_prefetch_desc(&tm_k.m16);
       tma_prefetch_desc(&tm_v.m16);
-      mbar_arrive_expect_tx(q_full, wk.n_own * C::kNch * 2048);
+      mbar_arrive_expect_tx(q_full, wk.n_own * C::kQKNch * 2048);
     }
     __syncwarp();
-    load_page_runs<C::kNch>(sQ, kChunkBytes, tm_q, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh, q_full);
+    load_page_runs<C::kQKNch>(sQ, kChunkBytes, tm_q, lane < wk.n_own ? wk.own_page(lane) : 0, wk.n_own, wk.bh,
+                              q_full);
     int pid_next = (n_steps > 0 && lane < min(NP, n_cols)) ? __ldg(col_pages + wk.e0 + lane) : 0;
     int k_issued = 0, v_issued = 0;
     for (int st = 0; st < n_steps; ++st) {
@@ -137,14 +145,14 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
         pid_next = lane < min(NP, n_cols - (st + 1) * NP) ? __ldg(col_pages + wk.e0 + (st + 1) * NP + lane) : 0;
       const int ks = st % KS, vs = st % VS;
       if (st >= KS && !__all_sync(0xffffffffu, mbar_wait(&k_empty[ks], ((st / KS) - 1) & 1, ab))) break;
-      if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kNch * 2048);
+      if (lane == 0) mbar_arrive_expect_tx(&k_full[ks], n * C::kQKNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(sK + ks * C::kStage, kFwdStageChunk, tm_k, pid, n, kv_bh, &k_full[ks]);
+      load_page_runs<C::kQKNch>(sK + ks * C::kKStage, kFwdStageChunk, tm_k, pid, n, kv_bh, &k_full[ks]);
       k_issued = st + 1;
       if (st >= VS && !__all_sync(0xffffffffu, mbar_wait(&v_empty[vs], ((st / VS) - 1) & 1, ab))) break;
       if (lane == 0) mbar_arrive_expect_tx(&v_full[vs], n * C::kNch * 2048);
       __syncwarp();
-      load_page_runs<C::kNch>(sV + vs * C::kStage, kFwdStageChunk, tm_v, pid, n, kv_bh, &v_full[vs]);
+      load_page_runs<C::kNch>(sV + vs * C::kVStage, kFwdStageChunk, tm_v, pid, n, kv_bh, &v_full[vs]);
       v_issued = st + 1;
     }
     // no copy may still be landing in shared memory when the CTA exits
@@ -167,7 +175,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       if (!__all_sync(0xffffffffu, w)) return false;
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
-      const uint64_t dv = sdesc_add(dv0, vs * C::kStage);
+      const uint64_t dv = sdesc_add(dv0, vs * C::kVStage);
 #pragma unroll
       for (int j = 0; j < NP; ++j)
         if (j < n)
@@ -188,12 +196,21 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       }
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
-      const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
-      const uint64_t dk = sdesc_add(dk0, ks * C::kStage);
+      const uint64_t dk = sdesc_add(dk0, ks * C::kKStage);
+      if constexpr (F8) {
+        // 32 E4M3 elements (32 bytes) of K per MMA
+        const uint32_t idesc_s = idesc_e4m3(128, 16 * n);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk)
-        umma_ss_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
-                  sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
+        for (int kk = 0; kk < D / 32; ++kk)
+          umma_ss_e4m3_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                         sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
+      } else {
+        const uint32_t idesc_s = idesc_bf16(128, 16 * n, false, false);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          umma_ss_w(tmem + 64 * b, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32),
+                    sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32), idesc_s, kk > 0 ? 1u : 0u);
+      }
       umma_commit_w(&s_full[b]);
       umma_commit_w(&k_empty[ks]);
       if (st >= 1 && !issue_pv(st - 1)) ok = false;
@@ -208,6 +225,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
     const uint32_t code = wk.row_code(row);
     const int seg = code < 8 ? static_cast<int>(code) : -1;
+    if constexpr (F8) sl2 *= __ldg(q_descale + wk.bh) * __ldg(k_descale + kv_bh);  // scores of the dequantised Q, K
     const uint64_t sl2x2 = f2_pack(sl2, sl2);
     float m_used = -INFINITY, l = 0.f;
     bool ok = true;
@@ -362,15 +380,17 @@ __global__ void fill_kernel(const int32_t* __restrict__ fill, int64_t n_bh, int6
   }
 }
 
-template <int D>
+template <int D, bool F8>
 cudaError_t launch_fwd_t(const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
-                         __nv_bfloat16* o, float* lse, cudaStream_t st) {
-  using C = FwdCfg<D>;
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+                         __nv_bfloat16* o, float* lse, const float* q_descale, const float* k_descale,
+                         cudaStream_t st) {
+  using C = FwdCfg<D, F8>;
+  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   if (e != cudaSuccess) return e;
   if (a.n_work == 0) return cudaSuccess;
-  fwd_kernel<D><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
-      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.heads, a.kv_group, a.err);
+  fwd_kernel<D, F8><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
+      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.heads, a.kv_group, q_descale,
+      k_descale, a.err);
   return cudaGetLastError();
 }
 
@@ -378,7 +398,14 @@ cudaError_t launch_fwd_t(const TmaPages& tq, const TmaPages& tk, const TmaPages&
 
 cudaError_t launch_fwd(int head_dim, const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
                        __nv_bfloat16* o, float* lse, cudaStream_t st) {
-  return head_dim == 128 ? launch_fwd_t<128>(tq, tk, tv, a, o, lse, st) : launch_fwd_t<64>(tq, tk, tv, a, o, lse, st);
+  return head_dim == 128 ? launch_fwd_t<128, false>(tq, tk, tv, a, o, lse, nullptr, nullptr, st)
+                         : launch_fwd_t<64, false>(tq, tk, tv, a, o, lse, nullptr, nullptr, st);
+}
+
+cudaError_t launch_fwd_e4m3(const TmaPages& tq8, const TmaPages& tk8, const TmaPages& tv, const TileArgs& a,
+                            const float* q_descale, const float* k_descale, __nv_bfloat16* o, float* lse,
+                            cudaStream_t st) {
+  return launch_fwd_t<128, true>(tq8, tk8, tv, a, o, lse, q_descale, k_descale, st);
 }
 
 cudaError_t launch_fill(int head_dim, const int32_t* fill, int64_t n, int64_t bh, int64_t slots,

@@ -51,6 +51,18 @@ struct TileArgs {
 cudaError_t launch_fwd(int head_dim, const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
                        __nv_bfloat16* o, float* lse, cudaStream_t st);
 
+// K1 with E4M3 Q and K (head_dim 128): tq8 / tk8 map the one-byte codes (128
+// per 128-byte row), S is scaled by q_descale[bh] * k_descale[kv_bh].
+cudaError_t launch_fwd_e4m3(const TmaPages& tq8, const TmaPages& tk8, const TmaPages& tv, const TileArgs& a,
+                            const float* q_descale, const float* k_descale, __nv_bfloat16* o, float* lse,
+                            cudaStream_t st);
+
+// Per-slice E4M3 quantisation of a [bh, rows, head_dim] bf16 tensor: amax of
+// each slice, codes = e4m3(x * (448 / amax)), descale = amax / 448 (1 for an
+// all-zero slice).  `descale` doubles as the amax scratch.
+cudaError_t launch_quantize_e4m3(const __nv_bfloat16* x, int64_t bh, int64_t elems_per_bh, uint8_t* x8,
+                                 float* descale, cudaStream_t st);
+
 // K2: delta[row] = sum_d dO[row, d] * O[row, d] over rows = batch*heads*q_slots.
 cudaError_t launch_delta(int head_dim, const __nv_bfloat16* o, const __nv_bfloat16* d_o, float* delta,
                          int64_t rows, cudaStream_t st);

@@ -168,6 +168,33 @@ int spattn_plan_set_graph_device(spattn_plan_t plan, const int64_t* row_ptr, con
 int spattn_fwd(const void* q, const void* k, const void* v, spattn_plan_t plan, void* o, float* lse,
                void* stream);
 
+/* FP8 (E4M3) quantisation of Q or K for spattn_fwd_fp8: x is a DEVICE bf16
+ * tensor [bh, rows, head_dim] (head_dim 64 or 128, 16-byte aligned), read
+ * as bh slices (one per batch*head).  Per slice, amax = max |x|; x8
+ * (DEVICE, [bh, rows, head_dim] one-byte E4M3 codes: 1 sign, 4 exponent bits
+ * with bias 7, 3 mantissa bits, largest finite 448) receives
+ * e4m3(x * (448 / amax)) rounded to nearest-even and saturated to +-448, and
+ * descale (DEVICE, [bh] fp32, 4-byte aligned) receives amax / 448 (1 for an
+ * all-zero slice); every step is one correctly rounded fp32 operation.
+ * Inputs must be finite.  Asynchronous on `stream` (four launches).  This
+ * is the quantised Q / K line of work that the KPage page lists next to the
+ * method (zhuanzhiai.com paper page), applied to the forward only. */
+int spattn_quantize_fp8(const void* x, int64_t bh, int64_t rows, int head_dim, void* x8, float* descale,
+                        void* stream);
+
+/* Forward with E4M3 Q and K (head_dim 128 only, else
+ * SPATTN_ERR_UNSUPPORTED): q8 [batch, heads, q_slots, 128] and k8
+ * [batch, kv_heads, kv_slots, 128] hold E4M3 codes, q_descale [batch*heads]
+ * and k_descale [batch*kv_heads] their per-slice scales (as written by
+ * spattn_quantize_fp8), v is bf16.  Computes exactly what spattn_fwd
+ * computes for the dequantised inputs q8 * q_descale and k8 * k_descale: S
+ * is a kind::f8f6f4 tensor-core product accumulated in fp32; P, V and O stay
+ * bf16 as in spattn_fwd, and LSE is that of the dequantised scores.  Same
+ * layouts, alignment, fill of rows without work and error codes as
+ * spattn_fwd. */
+int spattn_fwd_fp8(const void* q8, const void* k8, const float* q_descale, const float* k_descale, const void* v,
+                   spattn_plan_t plan, void* o, float* lse, void* stream);
+
 /* Backward: dQ, dK, dV given O and LSE from spattn_fwd and the loss
  * gradient dO.  Uses the plan's fp32 workspace for rowsum(dO * O) and the
  * plan's work-item counter of the persistent dK/dV kernel, so backward calls
