@@ -168,8 +168,6 @@ template <bool FILL>
 __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
   extern __shared__ uint8_t dp_smem[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(dp_smem);               // [kListCap]
-  uint64_t* mhi = keys + kListCap;                                      // [kListCap] segments 4..7
-  int32_t* mpage = reinterpret_cast<int32_t*>(mhi + kListCap);          // [kListCap]
   __shared__ int n_keys;
   const int64_t ti = blockIdx.x;
   const int32_t h = blockIdx.y;
@@ -219,22 +217,10 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
     }
   }
   if (threadIdx.x != 0) return;
-  // merge: one entry per page, eight 16-bit segment masks in two words (in
-  // place: the merged index never passes the read index)
-  int m = 0;
-  for (int i = 0; i < n;) {
-    const int32_t p = static_cast<int32_t>(keys[i] >> 20);
-    uint64_t mk[2] = {0, 0};
-    for (; i < n && static_cast<int32_t>(keys[i] >> 20) == p; ++i) {
-      const int sg = static_cast<int>((keys[i] >> 16) & 0xF);
-      mk[sg >> 2] |= static_cast<uint64_t>(keys[i] & 0xFFFFu) << (16 * (sg & 3));
-    }
-    mpage[m] = p;
-    keys[m] = mk[0];
-    mhi[m] = mk[1];
-    ++m;
-  }
-  // strided compaction (the host planner's rule) and output
+  // Merge (one entry per page, eight 16-bit segment masks in two words) and
+  // strided compaction (the host planner's rule) in one pass over the sorted
+  // keys.  The rule looks at the entries of pages p .. p+3 only, so a window
+  // of the next four merged entries suffices.
   const int64_t slot = static_cast<int64_t>(h) * a.n_tmpl + ti;
   const int64_t off = FILL ? (slot == 0 ? 0 : a.counts[slot - 1]) : 0;
   int64_t cnt = 0;
@@ -251,34 +237,58 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
     }
     ++cnt;
   };
-  for (int i = 0; i < m;) {
-    const int32_t p = mpage[i];
-    const int k = a.strided ? dp_sub_group(dp_fold(keys[i], mhi[i])) : -1;
+  int32_t wp[4];
+  uint64_t wlo[4], whi[4];
+  int wn = 0, ki = 0;
+  auto refill = [&]() {
+    while (wn < 4 && ki < n) {
+      const int32_t p = static_cast<int32_t>(keys[ki] >> 20);
+      uint64_t mk[2] = {0, 0};
+      for (; ki < n && static_cast<int32_t>(keys[ki] >> 20) == p; ++ki) {
+        const int sg = static_cast<int>((keys[ki] >> 16) & 0xF);
+        mk[sg >> 2] |= static_cast<uint64_t>(keys[ki] & 0xFFFFu) << (16 * (sg & 3));
+      }
+      wp[wn] = p;
+      wlo[wn] = mk[0];
+      whi[wn] = mk[1];
+      ++wn;
+    }
+  };
+  refill();
+  while (wn > 0) {
+    const int32_t p = wp[0];
+    const int k = a.strided ? dp_sub_group(dp_fold(wlo[0], whi[0])) : -1;
+    int used = 1;
     if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= a.col_slots) {
-      int j = i;
+      int j = 0;
       bool same = true;
-      while (j < m && mpage[j] <= p + 3) {
-        if (dp_sub_group(dp_fold(keys[j], mhi[j])) != k) {
+      while (j < wn && wp[j] <= p + 3) {
+        if (dp_sub_group(dp_fold(wlo[j], whi[j])) != k) {
           same = false;
           break;
         }
         ++j;
       }
-      if (same && j - i >= 2) {
+      if (same && j >= 2) {
         uint64_t mk[2] = {0, 0};
-        for (int x = i; x < j; ++x) {
-          const int jj = mpage[x] - p;
+        for (int x = 0; x < j; ++x) {
+          const int jj = wp[x] - p;
           for (int sg = 0; sg < kMaxSegments; ++sg)
-            mk[sg >> 2] |= (((sg < 4 ? keys[x] : mhi[x]) >> (16 * (sg & 3) + 4 * k)) & 0xFull)
+            mk[sg >> 2] |= (((sg < 4 ? wlo[x] : whi[x]) >> (16 * (sg & 3) + 4 * k)) & 0xFull)
                            << (16 * (sg & 3) + 4 * jj);
         }
         emit(~static_cast<int32_t>(16 * p + 4 * k), mk[0], mk[1]);
-        i = j;
-        continue;
+        used = j;
       }
     }
-    emit(p, keys[i], mhi[i]);
-    ++i;
+    if (used == 1) emit(p, wlo[0], whi[0]);
+    for (int x = used; x < wn; ++x) {
+      wp[x - used] = wp[x];
+      wlo[x - used] = wlo[x];
+      whi[x - used] = whi[x];
+    }
+    wn -= used;
+    refill();
   }
   if (!FILL) {
     a.counts[slot] = cnt;
@@ -371,8 +381,8 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     const int64_t nc = std::max<int64_t>(static_cast<int64_t>(H) * (d.tq.n + d.tk.n), 1);
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_counts), nc * sizeof(int64_t)));
     if (e != cudaSuccess) return SPATTN_ERR_OOM;
-    cudaFuncSetAttribute(dp_list<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 20);
-    cudaFuncSetAttribute(dp_list<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 20);
+    cudaFuncSetAttribute(dp_list<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 8);
+    cudaFuncSetAttribute(dp_list<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 8);
     d.ready = true;
   }
   // the plan keeps its own copy of the graph (inspection calls read it later)
@@ -416,7 +426,7 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     a.flag = flag;
     return a;
   };
-  const size_t smem = kListCap * 20;
+  const size_t smem = kListCap * 8;
   ListArgs la[2] = {args(true), args(false)};
   const PassTemplates* tt[2] = {&d.tq, &d.tk};
   WorkList* wls[2] = {&P->wq, &P->wk};
