@@ -217,11 +217,17 @@ size_t union_size(const std::vector<int32_t>& a, const std::vector<int32_t>& b) 
 // lists overlap most are packed together.  Greedy agglomeration: the pair of
 // clusters with the largest overlap (column groups they share, weighted by
 // the pages of each group) merges first, while the merged cluster holds at
-// most 8 pages and at most 4 groups (one work item).  Clusters left with room
+// most 8 pages and at most 8 groups (one work item).  Clusters left with room
 // are then filled in slot order under the same limits.
+//
+// A merge saves the same pairs (the overlap) whatever the sizes of the two
+// clusters, but a 4-page block merged with a 1-page edge block leaves a tile
+// that nothing larger than 3 pages can fill.  With two_phase, the first
+// round merges only clusters of like size (both at least one full block of
+// 4 pages, or both smaller), and a second round then merges freely.
 std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency& adj,
                                                const std::vector<int64_t>& src_heads,
-                                               const std::vector<OwnBlock>& blocks) {
+                                               const std::vector<OwnBlock>& blocks, bool two_phase) {
   const int32_t nb = static_cast<int32_t>(blocks.size());
   const int32_t ng = col.n_groups;
   const int64_t n_codes = static_cast<int64_t>(ng) * static_cast<int64_t>(src_heads.size());
@@ -264,7 +270,10 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
     while (parent[x] != x) x = parent[x] = parent[parent[x]];
     return x;
   };
+  constexpr int kFullBlock = kBlockRows / kPageRows;
+  bool like_sizes = two_phase;  // first round of the two-phase grouping
   auto fits = [&](int32_t a, int32_t b) {
+    if (like_sizes && (npg[a] >= kFullBlock) != (npg[b] >= kFullBlock)) return false;
     return npg[a] + npg[b] <= kTilePages && union_size(groups[a], groups[b]) <= static_cast<size_t>(kMaxSegments);
   };
   auto overlap = [&](int32_t a, int32_t b) {
@@ -299,29 +308,37 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
       cnt[r] = 0;
     }
   };
-  for (int32_t b = 0; b < nb; ++b) push_candidates(b, true);
-  while (!heap.empty()) {
-    const auto [w, nd, a, b] = heap.top();
-    heap.pop();
-    if (parent[a] != a || parent[b] != b || !fits(a, b)) continue;
-    const int64_t exact = overlap(a, b);
-    if (exact != w) {
-      if (exact > 0) heap.emplace(exact, nd, a, b);
-      continue;
+  for (int round = 0; round < (two_phase ? 2 : 1); ++round) {
+    if (round == 1) {
+      like_sizes = false;
+      for (int32_t b = 0; b < nb; ++b)
+        if (parent[b] == b && npg[b] < kTilePages) push_candidates(b, true);
+    } else {
+      for (int32_t b = 0; b < nb; ++b) push_candidates(b, true);
     }
-    // merge b into a
-    parent[b] = a;
-    npg[a] += npg[b];
-    std::vector<int32_t> u;
-    std::set_union(groups[a].begin(), groups[a].end(), groups[b].begin(), groups[b].end(), std::back_inserter(u));
-    groups[a].swap(u);
-    u.clear();
-    std::set_union(sig[a].begin(), sig[a].end(), sig[b].begin(), sig[b].end(), std::back_inserter(u));
-    sig[a].swap(u);
-    std::vector<int32_t>().swap(sig[b]);
-    members[a].insert(members[a].end(), members[b].begin(), members[b].end());
-    std::vector<int32_t>().swap(members[b]);
-    if (npg[a] < kTilePages) push_candidates(a, false);
+    while (!heap.empty()) {
+      const auto [w, nd, a, b] = heap.top();
+      heap.pop();
+      if (parent[a] != a || parent[b] != b || !fits(a, b)) continue;
+      const int64_t exact = overlap(a, b);
+      if (exact != w) {
+        if (exact > 0) heap.emplace(exact, nd, a, b);
+        continue;
+      }
+      // merge b into a
+      parent[b] = a;
+      npg[a] += npg[b];
+      std::vector<int32_t> u;
+      std::set_union(groups[a].begin(), groups[a].end(), groups[b].begin(), groups[b].end(), std::back_inserter(u));
+      groups[a].swap(u);
+      u.clear();
+      std::set_union(sig[a].begin(), sig[a].end(), sig[b].begin(), sig[b].end(), std::back_inserter(u));
+      sig[a].swap(u);
+      std::vector<int32_t>().swap(sig[b]);
+      members[a].insert(members[a].end(), members[b].begin(), members[b].end());
+      std::vector<int32_t>().swap(members[b]);
+      if (npg[a] < kTilePages) push_candidates(a, false);
+    }
   }
   // fill: clusters left with room, in slot order of their first block (a
   // cluster's root is its lowest block index)
@@ -576,11 +593,14 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
         // Per unit, the packing with fewer physical pairs (then fewer items).
         if (mode != 2) build_head(own, col, adj, u, src, slot_tiles, part[u], acc, touched);
         if (mode != 1) {
-          WorkList sim;
-          build_head(own, col, adj, u, src, pack_similar(col, adj, src, blocks), sim, acc, touched);
-          const bool better = mode == 2 || sim.physical_pairs < part[u].physical_pairs ||
-                              (sim.physical_pairs == part[u].physical_pairs && sim.work.size() < part[u].work.size());
-          if (better) part[u] = std::move(sim);
+          // one-round and two-round similarity grouping (the latter not for mode 2)
+          for (int two = 0; two < (mode == 2 ? 1 : 2); ++two) {
+            WorkList sim;
+            build_head(own, col, adj, u, src, pack_similar(col, adj, src, blocks, two == 1), sim, acc, touched);
+            const bool better = (mode == 2 && two == 0) || sim.physical_pairs < part[u].physical_pairs ||
+                                (sim.physical_pairs == part[u].physical_pairs && sim.work.size() < part[u].work.size());
+            if (better) part[u] = std::move(sim);
+          }
         }
         order_longest_first(part[u]);
       }
