@@ -52,7 +52,7 @@ WORKLOAD_TEXT = {
     "tiny": "tiny STA: 5x6x10 grid, 4x4x4 tiles, clamped 3x3x3 window",
 }
 KERNEL_FLOPS_PER_PAIR_D = {"fwd": 4, "dkdv": 8, "dq": 6}  # algorithmic GEMM flops per useful pair / D
-KERNEL_SOURCES = ["sm100.cuh", "tile.cuh", "fwd.cu", "bwd.cu"]
+KERNEL_SOURCES = ["sm100.cuh", "tile.cuh", "fwd.cu", "bwd.cu", "plan.cpp"]  # kernels and the lists they walk
 
 
 def load_peaks():
