@@ -149,9 +149,15 @@ struct OwnBlock {
   int npg = 0;
   int strided_group = -1;  // k of the strided page, else -1
   std::vector<int32_t> groups;  // distinct, ascending
+  int32_t only = -1;       // >= 0: the unit owns only the rows of this group
 };
 
-std::vector<OwnBlock> owned_blocks(const Side& s) {
+// The owned units of a side: its 64-slot blocks.  With split_groups, a block
+// whose rows belong to several groups becomes one unit per group (the block's
+// pages that hold rows of the group, owning only those rows), so that a tile
+// can run over one group's list only; a page shared by two units is then
+// computed by two work items that own disjoint rows.
+std::vector<OwnBlock> owned_blocks(const Side& s, bool split_groups = false) {
   const int per = kBlockRows / kPageRows;
   const bool strided = strided_enabled();
   std::vector<OwnBlock> out;
@@ -179,9 +185,34 @@ std::vector<OwnBlock> owned_blocks(const Side& s) {
       if (s.group[i] >= 0) b.groups.push_back(s.group[i]);
     std::sort(b.groups.begin(), b.groups.end());
     b.groups.erase(std::unique(b.groups.begin(), b.groups.end()), b.groups.end());
+    if (split_groups && b.strided_group < 0 && b.groups.size() > 1) {
+      for (int32_t g : b.groups) {
+        OwnBlock u;
+        u.groups = {g};
+        u.only = g;
+        for (int i = 0; i < b.npg; ++i) {
+          const int64_t p0 = static_cast<int64_t>(b.pages[i]) * kPageRows;
+          bool has = false;
+          for (int64_t x = p0; x < std::min<int64_t>(p0 + kPageRows, s.slots) && !has; ++x) has = s.group[x] == g;
+          if (has) u.pages[u.npg++] = b.pages[i];
+        }
+        out.push_back(std::move(u));
+      }
+      continue;
+    }
     out.push_back(std::move(b));
   }
   return out;
+}
+
+// Smallest group with a row on regular page p (-1 if none): the unit of that
+// group owns the page's padded rows when the page is split between units.
+int32_t first_group_of_page(const Side& s, int32_t p) {
+  int32_t m = -1;
+  const int64_t p0 = static_cast<int64_t>(p) * kPageRows;
+  for (int64_t x = p0; x < std::min<int64_t>(p0 + kPageRows, s.slots); ++x)
+    if (s.group[x] >= 0 && (m < 0 || s.group[x] < m)) m = s.group[x];
+  return m;
 }
 
 // Owned tiles in slot order: whole blocks appended while the tile holds at
@@ -227,7 +258,8 @@ size_t union_size(const std::vector<int32_t>& a, const std::vector<int32_t>& b) 
 // 4 pages, or both smaller), and a second round then merges freely.
 std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency& adj,
                                                const std::vector<int64_t>& src_heads,
-                                               const std::vector<OwnBlock>& blocks, bool two_phase) {
+                                               const std::vector<OwnBlock>& blocks, bool two_phase,
+                                               std::vector<std::vector<int32_t>>* only_out = nullptr) {
   const int32_t nb = static_cast<int32_t>(blocks.size());
   const int32_t ng = col.n_groups;
   const int64_t n_codes = static_cast<int64_t>(ng) * static_cast<int64_t>(src_heads.size());
@@ -360,11 +392,19 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
   }
   std::vector<std::vector<int32_t>> tiles;
   tiles.reserve(heads_of_tiles.size());
+  if (only_out) only_out->clear();
   for (int32_t r : heads_of_tiles) {
-    std::vector<int32_t> pages;
-    for (int32_t b : members[r]) pages.insert(pages.end(), blocks[b].pages, blocks[b].pages + blocks[b].npg);
-    std::sort(pages.begin(), pages.end());
+    std::vector<std::pair<int32_t, int32_t>> pg;  // (page reference, owned group or -1)
+    for (int32_t b : members[r])
+      for (int i = 0; i < blocks[b].npg; ++i) pg.emplace_back(blocks[b].pages[i], blocks[b].only);
+    std::sort(pg.begin(), pg.end());
+    std::vector<int32_t> pages, only;
+    for (const auto& x : pg) {
+      pages.push_back(x.first);
+      only.push_back(x.second);
+    }
     tiles.push_back(std::move(pages));
+    if (only_out) only_out->push_back(std::move(only));
   }
   return tiles;
 }
@@ -376,11 +416,13 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
 // a K/V head's group for the key-owned pass (entries carry j).
 void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t unit,
                 const std::vector<int64_t>& src_heads, const std::vector<std::vector<int32_t>>& tiles, WorkList& wl,
-                std::vector<uint64_t>& acc, std::vector<int64_t>& touched) {
+                std::vector<uint64_t>& acc, std::vector<int64_t>& touched,
+                const std::vector<std::vector<int32_t>>* only = nullptr) {
   const int64_t npc = col.n_pages;
   const bool strided = strided_enabled();
   int32_t rg[kTilePages * kPageRows];
-  for (const auto& tile : tiles) {
+  for (size_t ti = 0; ti < tiles.size(); ++ti) {
+    const auto& tile = tiles[ti];
     const int npg = static_cast<int>(tile.size());
     std::vector<int32_t> segs;
     for (int r = 0; r < kTilePages * kPageRows; ++r) {
@@ -388,6 +430,11 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       if (r < npg * kPageRows) {
         const int64_t slot = pref_slot(tile[r / kPageRows], r % kPageRows);
         if (slot < own.slots) g = own.group[slot];
+        const int32_t og = only ? (*only)[ti][r / kPageRows] : -1;
+        // a page split between units: this item owns the rows of its group,
+        // and the padded rows if its group is the page's smallest
+        if (og >= 0 && ((g >= 0 && g != og) || (g == -1 && og != first_group_of_page(own, tile[r / kPageRows]))))
+          g = -2;
       }
       rg[r] = g;
       if (g >= 0 && std::find(segs.begin(), segs.end(), g) == segs.end()) segs.push_back(g);
@@ -559,6 +606,7 @@ int packing_mode() {
   if (!env) return 0;
   if (std::strcmp(env, "slot") == 0) return 1;
   if (std::strcmp(env, "similar") == 0) return 2;
+  if (std::strcmp(env, "split") == 0) return 3;  // only the two-round grouping of group-split blocks
   return 0;
 }
 
@@ -571,6 +619,7 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
                    int32_t batch_copies, const std::function<std::vector<int64_t>(int32_t)>& src_heads,
                    WorkList& wl) {
   const auto blocks = owned_blocks(own);
+  const auto split_blocks = owned_blocks(own, true);
   const auto slot_tiles = pack_slot_order(blocks);
 
   const int mode = packing_mode();
@@ -591,13 +640,17 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
         const std::vector<int64_t> src = src_heads(u);
         acc.assign(static_cast<size_t>(col.n_pages) * src.size() * kMaskWords, 0);
         // Per unit, the packing with fewer physical pairs (then fewer items).
-        if (mode != 2) build_head(own, col, adj, u, src, slot_tiles, part[u], acc, touched);
+        if (mode == 0 || mode == 1) build_head(own, col, adj, u, src, slot_tiles, part[u], acc, touched);
         if (mode != 1) {
-          // one-round and two-round similarity grouping (the latter not for mode 2)
-          for (int two = 0; two < (mode == 2 ? 1 : 2); ++two) {
+          // one-round grouping of whole blocks (modes 0, 2), and two-round
+          // grouping of blocks split by group (modes 0, 3)
+          for (int two = (mode == 3 ? 1 : 0); two < (mode == 2 ? 1 : 2); ++two) {
             WorkList sim;
-            build_head(own, col, adj, u, src, pack_similar(col, adj, src, blocks, two == 1), sim, acc, touched);
-            const bool better = (mode == 2 && two == 0) || sim.physical_pairs < part[u].physical_pairs ||
+            std::vector<std::vector<int32_t>> only;
+            const auto tiles = pack_similar(col, adj, src, two == 1 ? split_blocks : blocks, two == 1, &only);
+            build_head(own, col, adj, u, src, tiles, sim, acc, touched, &only);
+            const bool forced = mode == 2 || mode == 3;
+            const bool better = forced || sim.physical_pairs < part[u].physical_pairs ||
                                 (sim.physical_pairs == part[u].physical_pairs && sim.work.size() < part[u].work.size());
             if (better) part[u] = std::move(sim);
           }

@@ -132,6 +132,18 @@ def test_tiny_full_parity(name, batch):
     check_tiny(p, t, out, batch)
 
 
+@pytest.mark.parametrize("batch", [1, 2])
+def test_tiny_split_packing_parity(batch, monkeypatch):
+    """Clustered layout with the group-split packing forced: pages shared by
+    two work items (each owning the rows of its cluster) in both passes."""
+    p = W.make_problem("tiny_svg2")
+    monkeypatch.setenv("SPATTN_PLAN_PACK", "split")
+    pl = sp.Plan.from_problem(p, batch=batch)
+    monkeypatch.delenv("SPATTN_PLAN_PACK")
+    t, out, _ = run_gpu(p, batch, pl=pl)
+    check_tiny(p, t, out, batch)
+
+
 def test_empty_column_lists_are_exercised():
     """tiny_nokeys head 1 attends nothing: its work items have empty column
     lists (no steps); the outputs are exact zeros and LSE = -inf there."""

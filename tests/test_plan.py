@@ -106,11 +106,30 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
     return pairs, owned
 
 
+def _split_pages(pl, which):
+    """Work items that repeat a page another item also owns rows of."""
+    work, _, _ = pl.work(which)
+    seen, shared = {}, 0
+    for w in work:
+        for r in w[4:4 + int(w[1])].tolist():
+            seen[(int(w[0]), r)] = seen.get((int(w[0]), r), 0) + 1
+    return sum(1 for v in seen.values() if v > 1)
+
+
 @pytest.mark.parametrize("name", TINY)
 @pytest.mark.parametrize("which", [0, 1])
-def test_coverage_invariant_tiny(name, which):
+@pytest.mark.parametrize("pack", ["best", "split"])
+def test_coverage_invariant_tiny(name, which, pack, monkeypatch):
+    """Every allowed pair exactly once, on exactly one owned row; with the
+    group-split packing forced, pages shared by several work items (each
+    owning the rows of its group) are covered exactly once as well."""
     p = W.make_problem(name)
+    if pack == "split":
+        monkeypatch.setenv("SPATTN_PLAN_PACK", "split")
     pl = sp.Plan.from_problem(p)
+    monkeypatch.delenv("SPATTN_PLAN_PACK", raising=False)
+    if pack == "split" and name == "tiny_svg2":
+        assert _split_pages(pl, which) > 0  # the clustered layout does split pages
     pairs, owned = _covered(p, pl, which)
     assert all(v == 1 for v in pairs.values()), "a pair is computed by two owned rows"
     own_group = p.q_group if which == 0 else p.kv_group
