@@ -150,7 +150,8 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
   a.heads = P->heads;
   a.kv_heads = P->kv_heads;
   a.kv_group = P->heads / P->kv_heads;
-  a.col_heads = w.d_heads;
+  // entry head offsets exist only under grouped-query attention (else all 0)
+  a.col_heads = P->kv_heads == P->heads ? nullptr : w.d_heads;
   return a;
 }
 
@@ -338,7 +339,6 @@ int spattn_plan_set_graph_device(spattn_plan_t plan, const int64_t* row_ptr, con
   if (!plan || !row_ptr || nnz < 0 || (nnz > 0 && !kv_groups)) return SPATTN_ERR_INVALID_ARG;
   const int st = check_plan_device(plan);
   if (st) return st;
-  if (plan->kv_heads != plan->heads || plan->graph_batches != 1) return SPATTN_ERR_UNSUPPORTED;
   try {
     return device_replan(plan, row_ptr, kv_groups, nnz, static_cast<cudaStream_t>(stream));
   } catch (...) {

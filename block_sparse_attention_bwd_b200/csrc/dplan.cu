@@ -151,41 +151,53 @@ struct ListArgs {
   const int32_t* gp_page;
   const uint16_t* gp_mask;
   int64_t col_slots;
-  int32_t heads, batch;
+  // units: grid y.  Unit u takes its columns from graph heads src(u, j),
+  // j < src_n: u itself in the query-owned pass (a graph head), the query
+  // heads of K/V head u % kv_heads of graph batch u / kv_heads in the
+  // key-owned pass.  Its items are repeated for `copies` batch entries
+  // (one graph for all of them), with work word 0 = copy * owned_heads + u.
+  int32_t n_units, src_n, heads, kv_heads, owned_heads, copies;
   bool strided;
   // outputs
-  int64_t* counts;          // [heads * n_tmpl] entries; inclusive-scanned between the passes
-  int32_t* out_work;        // [batch * heads * n_tmpl * 32] (fill pass)
+  int64_t* counts;          // [n_units * n_tmpl] entries; inclusive-scanned between the passes
+  int32_t* out_work;        // [copies * n_units * n_tmpl * 32] (fill pass)
   int32_t* out_pages;
   uint64_t* out_masks;
+  uint16_t* out_heads;      // entry head offsets j (key-owned pass under grouped-query attention) or null
   unsigned long long* stats;  // [0] useful pairs (one batch, query pass), [1 + pass] entries
   int pass;                   // 0 = query-owned, 1 = key-owned
   int* flag;
 };
 
-// One CTA per (template, head): the column list of that work item.
+// One CTA per (template, unit): the column list of that work item.
 template <bool FILL>
 __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
   extern __shared__ uint8_t dp_smem[];
   uint64_t* keys = reinterpret_cast<uint64_t*>(dp_smem);               // [kListCap]
   __shared__ int n_keys;
   const int64_t ti = blockIdx.x;
-  const int32_t h = blockIdx.y;
+  const int32_t u = blockIdx.y;
   if (threadIdx.x == 0) n_keys = 0;
   __syncthreads();
-  // gather (page << 20 | segment << 16 | row mask of the column group on the page)
-  for (int s = 0; s < kMaxSegments; ++s) {
-    const int32_t g = a.segs[ti * kMaxSegments + s];
-    if (g < 0) continue;
-    int64_t r0, r1;
-    dp_row(a.adj_ptr, static_cast<int64_t>(h) * a.n_src + g, a.adj_nnz, r0, r1, a.flag);
-    for (int64_t e = r0 + threadIdx.x; e < r1; e += blockDim.x) {
-      const int32_t b = a.adj_dst[e];
-      if (b < 0 || b >= a.n_col_groups) continue;
-      for (int64_t x = a.gp_ptr[b]; x < a.gp_ptr[b + 1]; ++x) {
-        const int idx = atomicAdd(&n_keys, 1);
-        if (idx < kListCap)
-          keys[idx] = (static_cast<uint64_t>(a.gp_page[x]) << 20) | (static_cast<uint64_t>(s) << 16) | a.gp_mask[x];
+  // gather (j << 44 | page << 20 | segment << 16 | row mask of the column
+  // group on the page), j the head offset of the source graph head
+  for (int j = 0; j < a.src_n; ++j) {
+    const int64_t gh = a.pass == 0 ? static_cast<int64_t>(u)
+                                   : static_cast<int64_t>(u / a.kv_heads) * a.heads + (u % a.kv_heads) * a.src_n + j;
+    for (int s = 0; s < kMaxSegments; ++s) {
+      const int32_t g = a.segs[ti * kMaxSegments + s];
+      if (g < 0) continue;
+      int64_t r0, r1;
+      dp_row(a.adj_ptr, gh * a.n_src + g, a.adj_nnz, r0, r1, a.flag);
+      for (int64_t e = r0 + threadIdx.x; e < r1; e += blockDim.x) {
+        const int32_t b = a.adj_dst[e];
+        if (b < 0 || b >= a.n_col_groups) continue;
+        for (int64_t x = a.gp_ptr[b]; x < a.gp_ptr[b + 1]; ++x) {
+          const int idx = atomicAdd(&n_keys, 1);
+          if (idx < kListCap)
+            keys[idx] = (static_cast<uint64_t>(j) << 44) | (static_cast<uint64_t>(a.gp_page[x]) << 20) |
+                        (static_cast<uint64_t>(s) << 16) | a.gp_mask[x];
+        }
       }
     }
   }
@@ -217,34 +229,36 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
     }
   }
   if (threadIdx.x != 0) return;
-  // Merge (one entry per page, eight 16-bit segment masks in two words) and
-  // strided compaction (the host planner's rule) in one pass over the sorted
-  // keys.  The rule looks at the entries of pages p .. p+3 only, so a window
-  // of the next four merged entries suffices.
-  const int64_t slot = static_cast<int64_t>(h) * a.n_tmpl + ti;
+  // Merge (one entry per (head offset, page), eight 16-bit segment masks in
+  // two words) and strided compaction (the host planner's rule) in one pass
+  // over the sorted keys.  The rule looks at the entries of pages p .. p+3 of
+  // one head offset only, so a window of the next four merged entries
+  // suffices.
+  const int64_t slot = static_cast<int64_t>(u) * a.n_tmpl + ti;
   const int64_t off = FILL ? (slot == 0 ? 0 : a.counts[slot - 1]) : 0;
   int64_t cnt = 0;
   unsigned long long useful = 0;
   const int32_t* sr = a.seg_rows + ti * kMaxSegments;
-  auto emit = [&](int32_t ref, uint64_t lo, uint64_t hi) {
+  auto emit = [&](int32_t ref, int32_t j, uint64_t lo, uint64_t hi) {
     if (FILL) {
       a.out_pages[off + cnt] = ref;
       a.out_masks[2 * (off + cnt)] = lo;
       a.out_masks[2 * (off + cnt) + 1] = hi;
+      if (a.out_heads) a.out_heads[off + cnt] = static_cast<uint16_t>(j);
     } else {
       for (int s = 0; s < kMaxSegments; ++s)
         useful += static_cast<unsigned long long>(sr[s]) * __popcll(((s < 4 ? lo : hi) >> (16 * (s & 3))) & 0xFFFFull);
     }
     ++cnt;
   };
-  int32_t wp[4];
+  int64_t wp[4];  // (head offset << 24) | page
   uint64_t wlo[4], whi[4];
   int wn = 0, ki = 0;
   auto refill = [&]() {
     while (wn < 4 && ki < n) {
-      const int32_t p = static_cast<int32_t>(keys[ki] >> 20);
+      const int64_t p = static_cast<int64_t>(keys[ki] >> 20);
       uint64_t mk[2] = {0, 0};
-      for (; ki < n && static_cast<int32_t>(keys[ki] >> 20) == p; ++ki) {
+      for (; ki < n && static_cast<int64_t>(keys[ki] >> 20) == p; ++ki) {
         const int sg = static_cast<int>((keys[ki] >> 16) & 0xF);
         mk[sg >> 2] |= static_cast<uint64_t>(keys[ki] & 0xFFFFu) << (16 * (sg & 3));
       }
@@ -256,13 +270,14 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
   };
   refill();
   while (wn > 0) {
-    const int32_t p = wp[0];
+    const int64_t jp = wp[0];
+    const int32_t p = static_cast<int32_t>(jp & 0xFFFFFF), jh = static_cast<int32_t>(jp >> 24);
     const int k = a.strided ? dp_sub_group(dp_fold(wlo[0], whi[0])) : -1;
     int used = 1;
     if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= a.col_slots) {
       int j = 0;
       bool same = true;
-      while (j < wn && wp[j] <= p + 3) {
+      while (j < wn && wp[j] <= jp + 3) {  // p + 3 stays below 2^24: the same head offset
         if (dp_sub_group(dp_fold(wlo[j], whi[j])) != k) {
           same = false;
           break;
@@ -272,16 +287,16 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
       if (same && j >= 2) {
         uint64_t mk[2] = {0, 0};
         for (int x = 0; x < j; ++x) {
-          const int jj = wp[x] - p;
+          const int jj = static_cast<int>(wp[x] - jp);
           for (int sg = 0; sg < kMaxSegments; ++sg)
             mk[sg >> 2] |= (((sg < 4 ? wlo[x] : whi[x]) >> (16 * (sg & 3) + 4 * k)) & 0xFull)
                            << (16 * (sg & 3) + 4 * jj);
         }
-        emit(~static_cast<int32_t>(16 * p + 4 * k), mk[0], mk[1]);
+        emit(~static_cast<int32_t>(16 * p + 4 * k), jh, mk[0], mk[1]);
         used = j;
       }
     }
-    if (used == 1) emit(p, wlo[0], whi[0]);
+    if (used == 1) emit(p, jh, wlo[0], whi[0]);
     for (int x = used; x < wn; ++x) {
       wp[x - used] = wp[x];
       wlo[x - used] = wlo[x];
@@ -296,10 +311,10 @@ __global__ void __launch_bounds__(kListThreads) dp_list(ListArgs a) {
     atomicAdd(&a.stats[1 + a.pass], static_cast<unsigned long long>(cnt));
   } else {
     const int32_t* tw = a.words + ti * 32;
-    for (int32_t b = 0; b < a.batch; ++b) {
-      int32_t* w = a.out_work + ((static_cast<int64_t>(b) * a.heads + h) * a.n_tmpl + ti) * 32;
+    for (int32_t b = 0; b < a.copies; ++b) {
+      int32_t* w = a.out_work + ((static_cast<int64_t>(b) * a.n_units + u) * a.n_tmpl + ti) * 32;
       for (int x = 0; x < 32; ++x) w[x] = tw[x];
-      w[0] = b * a.heads + h;
+      w[0] = b * a.owned_heads + u;
       w[2] = static_cast<int32_t>(off);
       w[3] = static_cast<int32_t>(off + cnt);
     }
@@ -356,7 +371,12 @@ void free_device_planner(DevPlanner& d) {
 int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_groups, int64_t nnz, cudaStream_t st) {
   DevPlanner& d = P->dp;
   const int32_t H = P->heads, nq = P->q.n_groups, nk = P->k.n_groups;
-  const int64_t rows_f = static_cast<int64_t>(H) * nq, rows_b = static_cast<int64_t>(H) * nk;
+  const int32_t kvh = P->kv_heads, grp = H / kvh, gb = P->graph_batches, copies = P->batch / gb;
+  const int32_t GH = gb * H;                   // graph heads (query-owned units)
+  const int32_t units[2] = {GH, gb * kvh};     // units of the query- and key-owned passes
+  const int64_t rows_f = static_cast<int64_t>(GH) * nq, rows_b = static_cast<int64_t>(GH) * nk;
+  // keys hold a page in 24 bits
+  if (P->q.n_pages >= (int64_t(1) << 24) || P->k.n_pages >= (int64_t(1) << 24)) return SPATTN_ERR_UNSUPPORTED;
   cudaError_t e = cudaSuccess;
   auto ck = [&](cudaError_t x) {
     if (e == cudaSuccess) e = x;
@@ -378,7 +398,7 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_cursor), std::max<int64_t>(rows_b, 1) * sizeof(int64_t)));
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_fwd_ptr), (rows_f + 1) * sizeof(int64_t)));
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_stats), 4 * sizeof(unsigned long long) + sizeof(int)));
-    const int64_t nc = std::max<int64_t>(static_cast<int64_t>(H) * (d.tq.n + d.tk.n), 1);
+    const int64_t nc = std::max<int64_t>(static_cast<int64_t>(units[0]) * d.tq.n + static_cast<int64_t>(units[1]) * d.tk.n, 1);
     ck(cudaMalloc(reinterpret_cast<void**>(&d.d_counts), nc * sizeof(int64_t)));
     if (e != cudaSuccess) return SPATTN_ERR_OOM;
     cudaFuncSetAttribute(dp_list<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kListCap * 8);
@@ -398,9 +418,9 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
   if (e != cudaSuccess) return SPATTN_ERR_CUDA;
   const unsigned g1 = static_cast<unsigned>(std::min<int64_t>((std::max(rows_f, nnz) + 255) / 256, 148 * 8));
   dp_validate<<<g1, 256, 0, st>>>(d.d_fwd_ptr, d.d_fwd_dst, rows_f, nnz, nk, flag);
-  dp_t_count<<<g1, 256, 0, st>>>(d.d_fwd_ptr, d.d_fwd_dst, H, nq, nk, nnz, d.d_bwd_ptr, flag);
+  dp_t_count<<<g1, 256, 0, st>>>(d.d_fwd_ptr, d.d_fwd_dst, GH, nq, nk, nnz, d.d_bwd_ptr, flag);
   dp_scan_inclusive<<<1, 1024, 0, st>>>(d.d_bwd_ptr + 1, rows_b);
-  dp_t_scatter<<<g1, 256, 0, st>>>(d.d_fwd_ptr, d.d_fwd_dst, H, nq, nk, nnz, d.d_bwd_ptr, d.d_cursor, d.d_bwd_dst, flag);
+  dp_t_scatter<<<g1, 256, 0, st>>>(d.d_fwd_ptr, d.d_fwd_dst, GH, nq, nk, nnz, d.d_bwd_ptr, d.d_cursor, d.d_bwd_dst, flag);
   const bool strided = strided_setting();
   auto args = [&](bool qpass) {
     ListArgs a;
@@ -418,8 +438,13 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     a.gp_page = qpass ? d.d_k_gp_page : d.d_q_gp_page;
     a.gp_mask = qpass ? d.d_k_gp_mask : d.d_q_gp_mask;
     a.col_slots = qpass ? P->k.slots : P->q.slots;
+    a.n_units = units[qpass ? 0 : 1];
+    a.src_n = qpass ? 1 : grp;
     a.heads = H;
-    a.batch = P->batch;
+    a.kv_heads = kvh;
+    a.owned_heads = qpass ? H : kvh;
+    a.copies = copies;
+    a.out_heads = nullptr;
     a.strided = strided;
     a.counts = d.d_counts;
     a.stats = stats;
@@ -434,11 +459,11 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
   // any list of the plan is touched (a rejected graph leaves the plan as it was)
   for (int pass = 0; pass < 2; ++pass) {
     la[pass].pass = pass;
-    la[pass].counts = d.d_counts + (pass == 0 ? 0 : static_cast<int64_t>(H) * d.tq.n);
-    if (tt[pass]->n > 0) {
-      dp_list<false><<<dim3(static_cast<unsigned>(tt[pass]->n), static_cast<unsigned>(H)), kListThreads, smem, st>>>(
-          la[pass]);
-      dp_scan_inclusive<<<1, 1024, 0, st>>>(la[pass].counts, static_cast<int64_t>(H) * tt[pass]->n);
+    la[pass].counts = d.d_counts + (pass == 0 ? 0 : static_cast<int64_t>(units[0]) * d.tq.n);
+    if (tt[pass]->n > 0 && units[pass] > 0) {
+      dp_list<false><<<dim3(static_cast<unsigned>(tt[pass]->n), static_cast<unsigned>(units[pass])), kListThreads, smem,
+                       st>>>(la[pass]);
+      dp_scan_inclusive<<<1, 1024, 0, st>>>(la[pass].counts, static_cast<int64_t>(units[pass]) * tt[pass]->n);
     }
   }
   if (cudaGetLastError() != cudaSuccess) return SPATTN_ERR_CUDA;
@@ -450,12 +475,12 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     return SPATTN_ERR_CUDA;
   if (hflag == kDpBadGraph) return SPATTN_ERR_INVALID_ARG;
   if (hflag == kDpOverflow) return SPATTN_ERR_UNSUPPORTED;
-  const int64_t useful = static_cast<int64_t>(hs[0]);
+  const int64_t useful = static_cast<int64_t>(hs[0]) * copies;
   for (int pass = 0; pass < 2; ++pass) {
     const int64_t total = static_cast<int64_t>(hs[1 + pass]);
     if (total > static_cast<int64_t>(INT32_MAX)) return SPATTN_ERR_UNSUPPORTED;
     WorkList& wl = *wls[pass];
-    const int64_t n_work = static_cast<int64_t>(P->batch) * H * tt[pass]->n;
+    const int64_t n_work = static_cast<int64_t>(copies) * units[pass] * tt[pass]->n;
     if (ensure(&wl.d_work, wl.cap_work, n_work * kWorkWords) != cudaSuccess ||
         ensure(&wl.d_pages, wl.cap_pages, total) != cudaSuccess ||
         ensure(&wl.d_masks, wl.cap_masks, total * kMaskWords) != cudaSuccess)
@@ -463,15 +488,20 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
     la[pass].out_work = wl.d_work;
     la[pass].out_pages = wl.d_pages;
     la[pass].out_masks = wl.d_masks;
-    if (tt[pass]->n > 0)
-      dp_list<true><<<dim3(static_cast<unsigned>(tt[pass]->n), static_cast<unsigned>(H)), kListThreads, smem, st>>>(
-          la[pass]);
+    // head offsets of the key-owned entries under grouped-query attention
+    if (pass == 1 && grp > 1) {
+      if (ensure(&wl.d_heads, wl.cap_heads, total) != cudaSuccess) return SPATTN_ERR_OOM;
+      la[pass].out_heads = wl.d_heads;
+    }
+    if (tt[pass]->n > 0 && units[pass] > 0)
+      dp_list<true><<<dim3(static_cast<unsigned>(tt[pass]->n), static_cast<unsigned>(units[pass])), kListThreads, smem,
+                      st>>>(la[pass]);
     if (cudaGetLastError() != cudaSuccess) return SPATTN_ERR_CUDA;
     wl.n_work = n_work;
     wl.n_entries_dev = total;
-    wl.physical_pairs = static_cast<int64_t>(kTilePages * kPageRows) * kPageRows * total * P->batch;
+    wl.physical_pairs = static_cast<int64_t>(kTilePages * kPageRows) * kPageRows * total * copies;
   }
-  P->useful_pairs = useful * P->batch;
+  P->useful_pairs = useful;
   P->bsa_pairs = -1;
   P->host_stale = true;
   P->graph_nnz = nnz;

@@ -852,6 +852,13 @@ int refresh_host(spattn_plan_s* P) {
                                          cudaMemcpyDeviceToHost) != cudaSuccess))
       return SPATTN_ERR_CUDA;
   }
+  // entry head offsets: written by the device planner under grouped-query
+  // attention, else all 0
+  P->wk.heads.assign(static_cast<size_t>(P->wk.n_entries_dev), 0);
+  if (P->kv_heads != P->heads && !P->wk.heads.empty() &&
+      cudaMemcpy(P->wk.heads.data(), P->wk.d_heads, P->wk.heads.size() * sizeof(uint16_t), cudaMemcpyDeviceToHost) !=
+          cudaSuccess)
+    return SPATTN_ERR_CUDA;
   const int64_t rows = static_cast<int64_t>(P->graph_batches) * P->heads * P->q.n_groups;
   std::vector<int64_t> rp(rows + 1);
   std::vector<int32_t> dst(std::max<int64_t>(P->graph_nnz, 1));
@@ -947,7 +954,7 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   if (P->device < 0) return SPATTN_OK;
 
   int64_t bytes = 0;
-  if ((st = upload(P->wk.heads, &P->wk.d_heads, bytes))) return st;
+  if ((st = upload(P->wk.heads, &P->wk.d_heads, bytes, &P->wk.cap_heads))) return st;
   for (WorkList* w : {&P->wq, &P->wk}) {
     if ((st = upload(w->work, &w->d_work, bytes, &w->cap_work))) return st;
     if ((st = upload(w->pages, &w->d_pages, bytes, &w->cap_pages))) return st;

@@ -72,7 +72,7 @@ struct WorkList {
   uint64_t* d_masks = nullptr;
   // capacities of the device arrays (elements) and, after a device re-plan,
   // the number of entries on the device
-  int64_t cap_work = 0, cap_pages = 0, cap_masks = 0;
+  int64_t cap_work = 0, cap_pages = 0, cap_masks = 0, cap_heads = 0;
   int64_t n_entries_dev = -1;
 };
 

@@ -145,9 +145,11 @@ int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_p
  * abstract evaluates, zhuanzhiai.com paper page) changes the graph every
  * call, and host planning of a large graph takes about a second; this call
  * rebuilds both work lists on the device in milliseconds.  row_ptr
- * ([heads * n_q_groups + 1]) and kv_groups ([nnz]) are DEVICE arrays in the
- * format of spattn_graph (rows may be unsorted and hold duplicates), read on
- * `stream`; the plan keeps its own copy.  The owned tiles are the layout's
+ * ([graph_batches * heads * n_q_groups + 1]) and kv_groups ([nnz]) are
+ * DEVICE arrays in the format of spattn_graph (rows may be unsorted and hold
+ * duplicates), read on `stream`; the plan keeps its own copy.  Grouped-query
+ * attention and per-batch graphs are handled as spattn_plan handles them
+ * (key-owned entries carry their query-head offset).  The owned tiles are the layout's
  * slot-order tiles (with strided pages); the column lists, strided entries,
  * pair counts and the transposed (key-owned) lists follow the new graph and
  * are identical to what spattn_plan would build with SPATTN_PLAN_PACK=slot,
@@ -155,7 +157,8 @@ int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_p
  * the new lists are used by every later spattn_fwd / spattn_bwd.  Returns
  * SPATTN_ERR_INVALID_ARG for a malformed graph (the plan is left unchanged),
  * SPATTN_ERR_UNSUPPORTED if one work item would gather more than 8192
- * (page, group) pairs, SPATTN_ERR_OOM if growing the plan's device lists
+ * (head, page, group) triples or a side has 2^24 pages or more,
+ * SPATTN_ERR_OOM if growing the plan's device lists
  * fails.  The inspection calls (stats, pages, qblocks, work) describe the
  * new graph (their first call copies it back to the host). */
 int spattn_plan_set_graph_device(spattn_plan_t plan, const int64_t* row_ptr, const int32_t* kv_groups, int64_t nnz,

@@ -7,6 +7,8 @@ backward passes on the re-planned lists must match the oracle; and a
 malformed graph must be rejected without touching the plan.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -19,13 +21,14 @@ pytestmark = pytest.mark.gpu
 
 
 def _items(plan, which):
-    """{(bh, owned refs, row codes): [(page ref, mask), ...]} of a work list."""
+    """{(bh, owned refs, row codes): [(page ref, mask, head offset), ...]} of a work list."""
     work, pages, masks = plan.work(which)
+    heads = plan.entry_heads(which)
     out = {}
     for w in work:
         n = int(w[1])
         key = (int(w[0]), tuple(int(x) for x in w[4:4 + n]), tuple(int(x) for x in w[12:28]))
-        lst = list(zip(pages[w[2]:w[3]].tolist(), map(tuple, masks[w[2]:w[3]].tolist())))
+        lst = list(zip(pages[w[2]:w[3]].tolist(), map(tuple, masks[w[2]:w[3]].tolist()), heads[w[2]:w[3]].tolist()))
         assert key not in out
         out[key] = lst
     return out
@@ -36,7 +39,7 @@ def _graph_variant(p, seed):
     (same lengths), from a seeded generator."""
     rng = np.random.default_rng(seed)
     rows = []
-    for r in range(p.heads * p.n_q_groups):
+    for r in range(p.graph_batches * p.heads * p.n_q_groups):
         n = int(p.row_ptr[r + 1] - p.row_ptr[r])
         rows.append(np.sort(rng.choice(p.n_kv_groups, size=min(n, p.n_kv_groups), replace=False)).tolist())
     row_ptr = np.zeros(len(rows) + 1, np.int64)
@@ -45,10 +48,11 @@ def _graph_variant(p, seed):
     return row_ptr, cols.astype(np.int32)
 
 
-def _host_slot_plan(p, row_ptr, cols, monkeypatch):
+def _host_slot_plan(p, row_ptr, cols, monkeypatch, batch=None):
     monkeypatch.setenv("SPATTN_PLAN_PACK", "slot")
-    pl = sp.Plan(p.q_group, p.kv_group, p.n_q_groups, p.n_kv_groups, row_ptr, cols, batch=p.batch, heads=p.heads,
-                 head_dim=p.head_dim, scale=p.scale)
+    pl = sp.Plan(p.q_group, p.kv_group, p.n_q_groups, p.n_kv_groups, row_ptr, cols,
+                 batch=p.batch if batch is None else batch, heads=p.heads, head_dim=p.head_dim, scale=p.scale,
+                 kv_heads=p.kv_heads, graph_batches=p.graph_batches)
     monkeypatch.delenv("SPATTN_PLAN_PACK")
     return pl
 
@@ -87,6 +91,30 @@ def test_device_replan_parity_tiny(name):
                   cols, p.seed_base)
     t, out, _ = run_gpu(q, pl=pl)
     check_tiny(q, t, out, 1)
+
+
+@pytest.mark.parametrize("name,batch", [("tiny_gqa", 2), ("tiny_mqa", 1), ("tiny_bgraph", 2)])
+def test_device_replan_grouped_heads_and_batch_graphs(name, batch, monkeypatch):
+    """Grouped-query attention (key-owned entries carry their query-head
+    offset) and one graph per batch entry: the re-planned lists equal the
+    host's slot-order plan of the same graph, entry heads included, and the
+    passes on them match the oracle."""
+    from test_gpu_parity import check_tiny, run_gpu
+
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p, batch=batch)
+    row_ptr, cols = _graph_variant(p, 23)
+    _replan(pl, row_ptr, cols)
+    ref = _host_slot_plan(p, row_ptr, cols, monkeypatch, batch=batch)
+    for which in (0, 1):
+        assert _items(pl, which) == _items(ref, which), which
+    a, b = pl.stats(), ref.stats()
+    for k in ("useful_pairs", "physical_pairs_fwd", "physical_pairs_dkdv", "n_work_fwd", "n_work_dkdv",
+              "n_entries_fwd", "n_entries_dkdv"):
+        assert a[k] == b[k], k
+    q = dataclasses.replace(p, row_ptr=row_ptr, kv_groups=cols)
+    t, out, _ = run_gpu(q, batch, pl=pl)
+    check_tiny(q, t, out, batch)
 
 
 def test_device_replan_rejects_bad_graph():
