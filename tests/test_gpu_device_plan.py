@@ -117,6 +117,30 @@ def test_device_replan_grouped_heads_and_batch_graphs(name, batch, monkeypatch):
     check_tiny(q, t, out, batch)
 
 
+@pytest.mark.parametrize("name,batch", [("tiny_vsa", 1), ("tiny_gqa", 2)])
+def test_device_replan_to_a_denser_graph(name, batch, monkeypatch):
+    """A dense graph re-planned over a sparse plan: every list grows past
+    the sizes the plan was built with (device buffers and per-entry arrays
+    must follow), and the passes on the new lists match the oracle."""
+    from test_gpu_parity import check_tiny, run_gpu
+
+    p = W.make_problem(name)
+    pl = sp.Plan.from_problem(p, batch=batch)
+    before = pl.stats()
+    rows = p.graph_batches * p.heads * p.n_q_groups
+    row_ptr = np.arange(rows + 1, dtype=np.int64) * p.n_kv_groups
+    cols = np.tile(np.arange(p.n_kv_groups, dtype=np.int32), rows)
+    _replan(pl, row_ptr, cols)
+    after = pl.stats()
+    assert after["n_entries_fwd"] > before["n_entries_fwd"] and after["n_entries_dkdv"] > before["n_entries_dkdv"]
+    ref = _host_slot_plan(p, row_ptr, cols, monkeypatch, batch=batch)
+    for which in (0, 1):
+        assert _items(pl, which) == _items(ref, which), which
+    q = dataclasses.replace(p, row_ptr=row_ptr, kv_groups=cols)
+    t, out, _ = run_gpu(q, batch, pl=pl)
+    check_tiny(q, t, out, batch)
+
+
 def test_device_replan_rejects_bad_graph():
     p = W.make_problem("tiny_vsa")
     t = {k: v.cuda() for k, v in W.make_tensors(p).items()}
