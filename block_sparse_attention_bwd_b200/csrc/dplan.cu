@@ -7,15 +7,18 @@
 // graph is rebuilt, on the device:
 //   * the owned tiles are the slot-order tiles of the layout (strided owned
 //     pages included), computed once on the host: for each tile and group
-//     split, a work item template (owned pages, row codes, the up-to-four
+//     split, a work item template (owned pages, row codes, the up-to-eight
 //     groups of its segments, the owned rows of each segment);
-//   * per (head, template) one CTA gathers, for each segment group, the
+//   * per (unit, template) one CTA gathers, for each segment group, the
 //     pages of every column group the graph lists for it (the column side's
 //     group -> page table), with the group's row mask on that page; sorts
-//     them by page in shared memory; merges them into one entry per page
-//     (eight 16-bit segment masks); and compacts runs of pages whose attended
-//     rows share a 4-row group into strided entries, exactly as the host
-//     planner does;
+//     them by (head offset, page) in shared memory; merges them into one
+//     entry per (head offset, page) (eight 16-bit segment masks); and
+//     compacts runs of pages whose attended rows share a 4-row group into
+//     strided entries, exactly as the host planner does.  A unit is a graph
+//     head in the query-owned pass and a (graph batch, K/V head) in the
+//     key-owned pass, whose columns come from every query head of its group
+//     (grouped-query attention; the entries carry the head offset);
 //   * the key-owned pass walks the transposed graph (key group -> query
 //     groups), built on the device with a counting sort;
 //   * two passes (count, then fill) with a device prefix sum place the lists.
