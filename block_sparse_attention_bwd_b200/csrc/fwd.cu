@@ -92,6 +92,8 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   const int kv_bh = (wk.bh / heads) * (heads / kv_group) + (wk.bh % heads) / kv_group;
   const int n_cols = wk.e1 - wk.e0;
   const int n_steps = (n_cols + NP - 1) / NP;
+  // 64-row route: every step holds two pages per half (a list of whole steps)
+  const bool halves = wk.halves() && (n_cols % NP) == 0;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
@@ -167,6 +169,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     const uint64_t dk0 = sdesc_sw128(smem_u32(sK), 16, 1024);
     const uint64_t dv0 = sdesc_sw128(smem_u32(sV), kFwdStageChunk, 1024);
     const uint32_t idesc_pv = idesc_bf16(128, D, false, true);
+    const uint32_t idesc_pv64 = idesc_bf16(64, D, false, true);
     bool ok = __all_sync(0xffffffffu, mbar_wait(q_full, 0, ab));
     tc_fence_after();
     auto issue_pv = [&](int st) -> bool {
@@ -176,10 +179,21 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
       const uint64_t dv = sdesc_add(dv0, vs * C::kVStage);
+      if (halves) {
+        // O_h += P_h V_h: half h's P (lanes from 16h) against the step's pages 2h, 2h+1
 #pragma unroll
-      for (int j = 0; j < NP; ++j)
-        if (j < n)
-          umma_ts_w(tO, tmem + 64 * b + 8 * j, sdesc_add(dv, j * 2048), idesc_pv, (st > 0 || j > 0) ? 1u : 0u);
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int j = 0; j < 2; ++j)
+            umma_ts_w(tO + (static_cast<uint32_t>(16 * h) << 16),
+                      tmem + 64 * b + (static_cast<uint32_t>(16 * h) << 16) + 8 * j,
+                      sdesc_add(dv, (2 * h + j) * 2048), idesc_pv64, (st > 0 || j > 0) ? 1u : 0u);
+      } else {
+#pragma unroll
+        for (int j = 0; j < NP; ++j)
+          if (j < n)
+            umma_ts_w(tO, tmem + 64 * b + 8 * j, sdesc_add(dv, j * 2048), idesc_pv, (st > 0 || j > 0) ? 1u : 0u);
+      }
       umma_commit_w(&v_empty[vs]);
       umma_commit_w(o_done);
       return true;
@@ -197,7 +211,29 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
       tc_fence_after();
       const int n = min(NP, n_cols - st * NP);
       const uint64_t dk = sdesc_add(dk0, ks * C::kKStage);
-      if constexpr (F8) {
+      if (halves) {
+        // S_h = Q_h K_h^T (M = 64, N = 32) for h = 0, 1: query rows 64h.. (8 KB
+        // into each chunk) against stage rows 32h.. (4 KB), written to the
+        // same 32 columns of buffer b at TMEM lanes offset by 16 h, so that
+        // row r of half h sits at lane 16 h + r % 16 + 32 (r / 16)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint32_t d = tmem + 64 * b + (static_cast<uint32_t>(16 * h) << 16);
+          if constexpr (F8) {
+#pragma unroll
+            for (int kk = 0; kk < D / 32; ++kk)
+              umma_ss_e4m3_w(d, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32 + h * 8192),
+                             sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32 + h * 4096), idesc_e4m3(64, 32),
+                             kk > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk)
+              umma_ss_w(d, sdesc_add(dq0, (kk >> 2) * kChunkBytes + (kk & 3) * 32 + h * 8192),
+                        sdesc_add(dk, (kk >> 2) * kFwdStageChunk + (kk & 3) * 32 + h * 4096),
+                        idesc_bf16(64, 32, false, false), kk > 0 ? 1u : 0u);
+          }
+        }
+      } else if constexpr (F8) {
         // 32 E4M3 elements (32 bytes) of K per MMA
         const uint32_t idesc_s = idesc_e4m3(128, 16 * n);
 #pragma unroll
@@ -221,8 +257,11 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   } else {
     // ---------------- softmax + epilogue (one row per thread) ----------------
     const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    // tile row of this thread's TMEM lane 32 q4 + lane: the lane itself, or
+    // in the 64-row route row (lane % 16) + 16 q4 of half hh
+    const int hh = (lane >> 4) & 1;
+    const int row = halves ? 64 * hh + (lane & 15) + 16 * q4 : q4 * 32 + lane;
     const uint32_t code = wk.row_code(row);
     const int seg = code < 8 ? static_cast<int>(code) : -1;
     if constexpr (F8) sl2 *= __ldg(q_descale + wk.bh) * __ldg(k_descale + kv_bh);  // scores of the dequantised Q, K
@@ -233,9 +272,11 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
     if (n_steps > 0) raw.fetch(col_masks, wk.e0, min(NP, n_cols), seg);
     for (int st = 0; st < n_steps; ++st) {
       const int b = st & 1;
-      const int N = 16 * min(NP, n_cols - st * NP);
+      // the 64-row route: 32 columns (this half's two pages) in the low half of S
+      const int N = halves ? 32 : 16 * min(NP, n_cols - st * NP);
       uint32_t mw[2];
       raw.bits(mw);
+      if (halves && hh) mw[0] = mw[1];
       // mask words of the next step load while this one computes
       if (st + 1 < n_steps) raw.fetch(col_masks, wk.e0 + (st + 1) * NP, min(NP, n_cols - (st + 1) * NP), seg);
       ok = __all_sync(0xffffffffu, mbar_wait(&s_full[b], (st >> 1) & 1, ab));

@@ -414,6 +414,62 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
 // before batch replication) whose columns come from the adjacency rows of the
 // graph heads src_heads[j]: one for the query-owned pass, the query heads of
 // a K/V head's group for the key-owned pass (entries carry j).
+// Column entries of one list, in slot order, from the masks accumulated in
+// `acc` for the (head offset, page) keys of `touched` (sorted); the keys' acc
+// words are cleared on the way.  Up to four consecutive pages whose attended
+// rows (over all segments) lie in one 4-row group k, at least two of them in
+// the list, become one strided entry: the four groups then cost one 16-column
+// page instead of one page each.
+void append_entries(const Side& col, bool strided, std::vector<uint64_t>& acc, const std::vector<int64_t>& touched,
+                    std::vector<int32_t>& pages, std::vector<uint64_t>& masks, std::vector<uint16_t>& heads) {
+  const int64_t npc = col.n_pages;
+  auto fold = [&](int64_t c) {
+    const uint64_t m = acc[2 * c] | acc[2 * c + 1];
+    return static_cast<uint32_t>((m | (m >> 16) | (m >> 32) | (m >> 48)) & 0xFFFFu);
+  };
+  size_t i = 0;
+  while (i < touched.size()) {
+    const int64_t c = touched[i];
+    const int32_t p = static_cast<int32_t>(c % npc);
+    const uint16_t jh = static_cast<uint16_t>(c / npc);
+    const int k = strided ? sub_group(fold(c)) : -1;
+    // (the bound keeps p + 3 inside the side, so c + 3 stays in head jh)
+    if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= col.slots) {
+      size_t j = i;
+      bool same = true;
+      while (j < touched.size() && touched[j] <= c + 3) {
+        if (sub_group(fold(touched[j])) != k) {
+          same = false;
+          break;
+        }
+        ++j;
+      }
+      if (same && j - i >= 2) {
+        uint64_t m[kMaskWords] = {0, 0};
+        for (size_t x = i; x < j; ++x) {
+          const int jj = static_cast<int>(touched[x] - c);
+          for (int sg = 0; sg < kMaxSegments; ++sg)
+            m[sg / 4] |= ((acc[2 * touched[x] + sg / 4] >> (16 * (sg % 4) + 4 * k)) & 0xFull)
+                         << (16 * (sg % 4) + 4 * jj);
+          acc[2 * touched[x]] = acc[2 * touched[x] + 1] = 0;
+        }
+        pages.push_back(~static_cast<int32_t>(16 * p + 4 * k));
+        masks.push_back(m[0]);
+        masks.push_back(m[1]);
+        heads.push_back(jh);
+        i = j;
+        continue;
+      }
+    }
+    pages.push_back(p);
+    masks.push_back(acc[2 * c]);
+    masks.push_back(acc[2 * c + 1]);
+    heads.push_back(jh);
+    acc[2 * c] = acc[2 * c + 1] = 0;
+    ++i;
+  }
+}
+
 void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t unit,
                 const std::vector<int64_t>& src_heads, const std::vector<std::vector<int32_t>>& tiles, WorkList& wl,
                 std::vector<uint64_t>& acc, std::vector<int64_t>& touched,
@@ -463,55 +519,7 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       w[0] = unit;
       w[1] = npg;
       w[2] = static_cast<int32_t>(wl.pages.size());
-      // Column entries in slot order.  Up to four consecutive pages whose
-      // attended rows (over all segments) lie in one 4-row group k, at least
-      // two of them in the list, become one strided entry: the four groups
-      // then cost one 16-column page instead of one page each.
-      auto fold = [&](int64_t c) {
-        const uint64_t m = acc[2 * c] | acc[2 * c + 1];
-        return static_cast<uint32_t>((m | (m >> 16) | (m >> 32) | (m >> 48)) & 0xFFFFu);
-      };
-      size_t i = 0;
-      while (i < touched.size()) {
-        const int64_t c = touched[i];
-        const int32_t p = static_cast<int32_t>(c % npc);
-        const uint16_t jh = static_cast<uint16_t>(c / npc);
-        const int k = strided ? sub_group(fold(c)) : -1;
-        // (the bound keeps p + 3 inside the side, so c + 3 stays in head jh)
-        if (k >= 0 && 16 * (static_cast<int64_t>(p) + 3) + 4 * k + 4 <= col.slots) {
-          size_t j = i;
-          bool same = true;
-          while (j < touched.size() && touched[j] <= c + 3) {
-            if (sub_group(fold(touched[j])) != k) {
-              same = false;
-              break;
-            }
-            ++j;
-          }
-          if (same && j - i >= 2) {
-            uint64_t m[kMaskWords] = {0, 0};
-            for (size_t x = i; x < j; ++x) {
-              const int jj = static_cast<int>(touched[x] - c);
-              for (int sg = 0; sg < kMaxSegments; ++sg)
-                m[sg / 4] |= ((acc[2 * touched[x] + sg / 4] >> (16 * (sg % 4) + 4 * k)) & 0xFull)
-                             << (16 * (sg % 4) + 4 * jj);
-              acc[2 * touched[x]] = acc[2 * touched[x] + 1] = 0;
-            }
-            wl.pages.push_back(~static_cast<int32_t>(16 * p + 4 * k));
-            wl.masks.push_back(m[0]);
-            wl.masks.push_back(m[1]);
-            wl.heads.push_back(jh);
-            i = j;
-            continue;
-          }
-        }
-        wl.pages.push_back(p);
-        wl.masks.push_back(acc[2 * c]);
-        wl.masks.push_back(acc[2 * c + 1]);
-        wl.heads.push_back(jh);
-        acc[2 * c] = acc[2 * c + 1] = 0;
-        ++i;
-      }
+      append_entries(col, strided, acc, touched, wl.pages, wl.masks, wl.heads);
       const size_t n_entries = wl.pages.size() - static_cast<size_t>(w[2]);
       w[3] = static_cast<int32_t>(wl.pages.size());
       for (int i = 0; i < npg; ++i) w[4 + i] = tile[i];
@@ -529,6 +537,115 @@ void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t 
       wl.work.insert(wl.work.end(), w, w + kWorkWords);
     }
   }
+}
+
+// Work items of the 64-row route (the KPage abstract's routing of Q blocks
+// to a smaller tile shape, B200 form): two 64-slot blocks per item, rows
+// 0..63 (owned pages 0..3) and 64..127 (owned pages 4..7), each half with
+// its own column list.  The forward runs each half as M = 64 products, so a
+// pair of blocks with unrelated lists (VSA-style selection) no longer pays
+// for the union of both lists.  The lists are interleaved two entries at a
+// time and padded to whole 4-entry steps with zero-mask entries (that repeat
+// a page of the list, so every load stays inside the tensor).  Blocks are
+// paired in slot order; a last odd block runs alone (its other half owns no
+// row).  Returns false, leaving wl partly built, when a pair holds more than
+// kMaxSegments groups.
+bool build_head_halves(const Side& own, const Side& col, const Adjacency& adj, int32_t unit,
+                       const std::vector<int64_t>& src_heads, const std::vector<OwnBlock>& blocks, WorkList& wl,
+                       std::vector<uint64_t>& acc, std::vector<int64_t>& touched) {
+  const int64_t npc = col.n_pages;
+  const bool strided = strided_enabled();
+  constexpr int kHalfPages = kTilePages / 2;
+  std::vector<int32_t> hp[2];
+  std::vector<uint64_t> hm[2];
+  std::vector<uint16_t> hh[2];
+  for (size_t bi = 0; bi < blocks.size(); bi += 2) {
+    const OwnBlock* half[2] = {&blocks[bi], bi + 1 < blocks.size() ? &blocks[bi + 1] : nullptr};
+    int32_t tile[kTilePages];
+    int32_t rg[kTilePages * kPageRows];  // segment of each row, or -1 (owned padded row) / -2 (not owned)
+    // Segments are numbered per half (those of half 0 first): a group with
+    // rows in both halves gets one segment in each, so that the entries of
+    // one half never carry bits of the other half's rows (a kernel that
+    // ignores the route then still computes every pair once).
+    std::vector<int32_t> segs;
+    size_t seg0[3] = {0, 0, 0};  // half h owns segments seg0[h] .. seg0[h+1]-1
+    for (int h = 0; h < 2; ++h) {
+      const OwnBlock* b = half[h] ? half[h] : half[0];
+      if (b->npg > kHalfPages) return false;
+      for (int i = 0; i < kHalfPages; ++i) tile[kHalfPages * h + i] = i < b->npg ? b->pages[i] : b->pages[0];
+      seg0[h] = segs.size();
+      for (int r = 64 * h; r < 64 * h + 64; ++r) {
+        int32_t g = -2;  // row not owned: a padding page, or beyond the tensor
+        if (half[h] && (r - 64 * h) / kPageRows < half[h]->npg) {
+          const int64_t slot = pref_slot(tile[r / kPageRows], r % kPageRows);
+          if (slot < own.slots) g = own.group[slot];
+        }
+        if (g < 0) {
+          rg[r] = g;
+          continue;
+        }
+        const auto first = segs.begin() + static_cast<std::ptrdiff_t>(seg0[h]);
+        const auto it = std::find(first, segs.end(), g);
+        rg[r] = static_cast<int32_t>(it - segs.begin());
+        if (it == segs.end()) segs.push_back(g);
+      }
+      seg0[h + 1] = segs.size();
+    }
+    if (segs.size() > static_cast<size_t>(kMaxSegments)) return false;
+    for (int h = 0; h < 2; ++h) {
+      touched.clear();
+      for (size_t j = 0; j < src_heads.size(); ++j)
+        for (int sg = static_cast<int>(seg0[h]); sg < static_cast<int>(seg0[h + 1]); ++sg) {
+          const int64_t r = src_heads[j] * adj.n_src + segs[sg];
+          for (int64_t e = adj.ptr[r]; e < adj.ptr[r + 1]; ++e) {
+            const int32_t b = adj.dst[e];
+            for (int64_t x = col.gp_ptr[b]; x < col.gp_ptr[b + 1]; ++x) {
+              const int64_t c = static_cast<int64_t>(j) * npc + col.gp_page[x];
+              if (acc[2 * c] == 0 && acc[2 * c + 1] == 0) touched.push_back(c);
+              acc[2 * c + sg / 4] |= static_cast<uint64_t>(col.gp_mask[x]) << (16 * (sg % 4));
+            }
+          }
+        }
+      std::sort(touched.begin(), touched.end());
+      hp[h].clear();
+      hm[h].clear();
+      hh[h].clear();
+      append_entries(col, strided, acc, touched, hp[h], hm[h], hh[h]);
+    }
+    int32_t w[kWorkWords];
+    std::memset(w, 0, sizeof(w));
+    w[0] = unit;
+    w[1] = kTilePages;
+    w[2] = static_cast<int32_t>(wl.pages.size());
+    const size_t n_steps = std::max((hp[0].size() + 1) / 2, (hp[1].size() + 1) / 2);
+    for (size_t st = 0; st < n_steps; ++st)
+      for (int h = 0; h < 2; ++h)
+        for (size_t j = 0; j < 2; ++j) {
+          const size_t idx = 2 * st + j;
+          if (idx < hp[h].size()) {
+            wl.pages.push_back(hp[h][idx]);
+            wl.masks.push_back(hm[h][2 * idx]);
+            wl.masks.push_back(hm[h][2 * idx + 1]);
+            wl.heads.push_back(hh[h][idx]);
+          } else {
+            wl.pages.push_back(!hp[h].empty() ? hp[h][0] : hp[1 - h][0]);
+            wl.masks.push_back(0);
+            wl.masks.push_back(0);
+            wl.heads.push_back(0);
+          }
+        }
+    w[3] = static_cast<int32_t>(wl.pages.size());
+    for (int i = 0; i < kTilePages; ++i) w[4 + i] = tile[i];
+    for (int r = 0; r < kTilePages * kPageRows; ++r) {
+      const uint32_t code = rg[r] >= 0 ? static_cast<uint32_t>(rg[r]) : (rg[r] == -1 ? kCodeNoSegment : kCodeNotOwned);
+      reinterpret_cast<uint32_t*>(w)[12 + r / 8] |= code << (4 * (r % 8));
+    }
+    w[28] = 1;
+    // each entry meets the 64 rows of its half
+    wl.physical_pairs += static_cast<int64_t>(64) * kPageRows * static_cast<int64_t>(w[3] - w[2]);
+    wl.work.insert(wl.work.end(), w, w + kWorkWords);
+  }
+  return true;
 }
 
 // Work item templates of the slot-order tiles (the device planner's items):
@@ -598,16 +715,41 @@ void order_longest_first(WorkList& w) {
   w.work.swap(out);
 }
 
-// Tile packing of a pass: 0 = best of the two per head (default), 1 = slot
-// order only, 2 = similarity grouping only.  SPATTN_PLAN_PACK=slot|similar
-// selects one (for comparisons and tests).
+// Tile packing of a pass: 0 = best per head (default), 1 = slot order only,
+// 2 = similarity grouping only, 3 = only the two-round grouping of
+// group-split blocks, 4 = the 64-row route for the query-owned pass wherever
+// a pair of blocks allows it (the key-owned pass as in 0).
+// SPATTN_PLAN_PACK=slot|similar|split|route64 selects one (for comparisons
+// and tests).
 int packing_mode() {
   const char* env = std::getenv("SPATTN_PLAN_PACK");
   if (!env) return 0;
   if (std::strcmp(env, "slot") == 0) return 1;
   if (std::strcmp(env, "similar") == 0) return 2;
-  if (std::strcmp(env, "split") == 0) return 3;  // only the two-round grouping of group-split blocks
+  if (std::strcmp(env, "split") == 0) return 3;
+  if (std::strcmp(env, "route64") == 0) return 4;
   return 0;
+}
+
+// Modelled time of a query-owned work list (forward then dQ, which both run
+// it), in forward steps of 128 rows x 64 columns.  A dQ step costs about
+// 1.45 forward steps whatever the route (dQ computes every entry against all
+// 128 rows).  A forward step of the 64-row route (2 x 64 rows x 32 columns)
+// costs 0.89-0.94 of one (measured on B200 with the route forced: partial
+// and VSA-style workloads): half the exponentials per row, but two M = 64
+// score products at N = 32 take as much tensor time as one M = 128 product
+// at N = 64.  So the route wins only where a tile's two blocks have
+// disjoint lists of equal length, which the workloads measured here never
+// give (the VSA-style union carries fewer steps than the padded halves).
+constexpr double kDqStepCost = 1.45;
+constexpr double kRoute64StepCost = 0.92;
+double query_pass_cost(const WorkList& w) {
+  double t = 0.0;
+  for (size_t i = 0; i < w.work.size(); i += kWorkWords) {
+    const int32_t* x = w.work.data() + i;
+    t += static_cast<double>((x[3] - x[2] + 3) / 4) * ((x[28] ? kRoute64StepCost : 1.0) + kDqStepCost);
+  }
+  return t;
 }
 
 // Work list of one pass.  Unit u (0 <= u < n_units) owns tensor head u of the
@@ -617,12 +759,13 @@ int packing_mode() {
 // their owned head shifted by b * owned_heads (they share the entries).
 int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32_t n_units, int32_t owned_heads,
                    int32_t batch_copies, const std::function<std::vector<int64_t>(int32_t)>& src_heads,
-                   WorkList& wl) {
+                   bool route64, WorkList& wl) {
   const auto blocks = owned_blocks(own);
   const auto split_blocks = owned_blocks(own, true);
   const auto slot_tiles = pack_slot_order(blocks);
 
-  const int mode = packing_mode();
+  const int route_mode = packing_mode();
+  const int mode = route_mode == 4 ? 0 : route_mode;  // tile packing of the 128-row route
   // Units are independent: each is built on its own into part[u] (worker t
   // takes units t, t + n, ...), then the parts are joined in unit order, so
   // the result does not depend on the number of threads.
@@ -654,6 +797,13 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
                                 (sim.physical_pairs == part[u].physical_pairs && sim.work.size() < part[u].work.size());
             if (better) part[u] = std::move(sim);
           }
+        }
+        // the 64-row route, where the model gives it the shorter time
+        if (route64 && (route_mode == 0 || route_mode == 4)) {
+          WorkList hv;
+          if (build_head_halves(own, col, adj, u, src, blocks, hv, acc, touched) &&
+              (route_mode == 4 || query_pass_cost(hv) < query_pass_cost(part[u])))
+            part[u] = std::move(hv);
         }
         order_longest_first(part[u]);
       }
@@ -929,7 +1079,7 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
 
   // query-owned pass: unit = graph head (its own graph rows)
   st = build_worklist(P->q, P->k, P->fwd_adj, GH, L->heads, copies,
-                      [](int32_t u) { return std::vector<int64_t>{u}; }, P->wq);
+                      [](int32_t u) { return std::vector<int64_t>{u}; }, true, P->wq);
   if (st) return st;
   // key-owned pass: unit = K/V head of a graph batch; its columns are the
   // transposed rows of the query heads of its group (head offset j)
@@ -942,7 +1092,7 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
                           v[j] = static_cast<int64_t>(u / kv_heads) * H + (u % kv_heads) * grp + j;
                         return v;
                       },
-                      P->wk);
+                      false, P->wk);
   if (st) return st;
 
   fill_list(P->q, P->q_fill);

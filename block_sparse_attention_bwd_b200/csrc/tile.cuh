@@ -33,6 +33,12 @@ struct Work {
   __device__ __forceinline__ uint32_t row_code(int r) const {
     return (static_cast<uint32_t>(w[12 + (r >> 3)]) >> (4 * (r & 7))) & 0xFu;
   }
+  // 64-row route (query-owned items only): rows 0..63 (own pages 0..3) and
+  // 64..127 (own pages 4..7) each run over their own pages, two per half in
+  // every 4-entry step (entries 0, 1 for rows 0..63, entries 2, 3 for the
+  // rest).  The masks alone already make the item exact, so a kernel that
+  // ignores the flag computes the same result over all 128 rows.
+  __device__ __forceinline__ bool halves() const { return w[28] != 0; }
 };
 
 __device__ __forceinline__ Work load_work(const int32_t* work, int64_t idx) {

@@ -279,6 +279,13 @@ int spattn_plan_qblocks(spattn_plan_t plan, int32_t head, int64_t page, const in
  *   [4..11] owned page references   [12..27] 128 row codes, 4 bits each,
  *   row r in word 12 + r/8 at bit 4*(r%8): 0..7 = segment, 14 = owned row
  *   with no segment (padded), 15 = row not written by this item.
+ *   [28] route of a query-owned item: 0 = all 128 rows run over the whole
+ *   list (entries in ascending slot order); 1 = 64-row route (the KPage
+ *   abstract's routing of Q blocks to smaller tiles): rows 0..63 (owned
+ *   pages 0..3) and rows 64..127 (owned pages 4..7) each have their own list,
+ *   interleaved two entries at a time (entries 4i, 4i+1 for rows 0..63,
+ *   4i+2, 4i+3 for rows 64..127, each half ascending; padding entries have
+ *   zero masks), so the entry count is a multiple of 4.  [29..31] zero.
  * A page reference p >= 0 is the page of slots 16p .. 16p+15; a negative
  * value is a strided page with base slot b = ~value, whose row r is slot
  * b + 16 (r / 4) + r % 4.  pages[e] is a page reference of the other side;

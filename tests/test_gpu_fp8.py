@@ -61,12 +61,18 @@ def test_quantize_bit_exact_wide_range():
     _check_quant(torch.randn(1, 2, 40, 64, generator=g).to(torch.bfloat16))
 
 
-@pytest.mark.parametrize("name,batch", [("tiny_d128", 1), ("tiny_vsa", 1), ("tiny_hedge", 1), ("tiny_svg2", 2),
-                                        ("tiny_gqa", 2), ("tiny_empty", 1), ("tiny_bgraph", 2)])
-def test_fwd_fp8_tiny_parity(name, batch):
+@pytest.mark.parametrize("name,batch,route", [("tiny_d128", 1, ""), ("tiny_vsa", 1, ""), ("tiny_hedge", 1, ""),
+                                              ("tiny_svg2", 2, ""), ("tiny_gqa", 2, ""), ("tiny_empty", 1, ""),
+                                              ("tiny_bgraph", 2, ""), ("tiny_vsa", 1, "route64"),
+                                              ("tiny_svg2", 2, "route64")])
+def test_fwd_fp8_tiny_parity(name, batch, route, monkeypatch):
     p = _d128(name) if name != "tiny_d128" else W.make_problem(name)
     t = W.make_tensors(p, batch=batch)
+    if route:
+        monkeypatch.setenv("SPATTN_PLAN_PACK", route)  # the 64-row route forced on every query-owned item
     pl = sp.Plan.from_problem(p, batch=batch)
+    monkeypatch.delenv("SPATTN_PLAN_PACK", raising=False)
+    assert (pl.work(0)[0][:, 28] == 1).all() or not route
     q8c, qd = _check_quant(t["q"])
     k8c, kd = _check_quant(t["k"])
     q8, qds = sp.quantize_fp8(t["q"].cuda())

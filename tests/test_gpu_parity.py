@@ -144,6 +144,22 @@ def test_tiny_split_packing_parity(batch, monkeypatch):
     check_tiny(p, t, out, batch)
 
 
+@pytest.mark.parametrize("name,batch", [(n, 1) for n in ["tiny", "tiny_vsa", "tiny_svg2", "tiny_hedge", "tiny_onekey",
+                                                          "tiny_nokeys", "tiny_d128", "tiny_gqa"]]
+                         + [("tiny_vsa", 2), ("tiny_bgraph", 2)])
+def test_tiny_route64_parity(name, batch, monkeypatch):
+    """The 64-row route forced on every query-owned item (two M = 64 halves
+    per tile, each over its own column list; dQ runs the same list over all
+    128 rows), forward and backward against the oracle."""
+    p = W.make_problem(name)
+    monkeypatch.setenv("SPATTN_PLAN_PACK", "route64")
+    pl = sp.Plan.from_problem(p, batch=batch)
+    monkeypatch.delenv("SPATTN_PLAN_PACK")
+    assert (pl.work(0)[0][:, 28] == 1).all()
+    t, out, _ = run_gpu(p, batch, pl=pl)
+    check_tiny(p, t, out, batch)
+
+
 def test_empty_column_lists_are_exercised():
     """tiny_nokeys head 1 attends nothing: its work items have empty column
     lists (no steps); the outputs are exact zeros and LSE = -inf there."""

@@ -78,11 +78,22 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
             continue
         n_own, e0, e1 = int(w[1]), int(w[2]), int(w[3])
         assert 1 <= n_own <= 8 and 0 <= e0 <= e1 <= pages.size and masks.shape == (pages.size, 2)
+        assert np.all(w[29:32] == 0) and int(w[28]) in (0, 1)
+        route = int(w[28]) == 1
         codes = _codes(w)
         pg = pages[e0:e1].astype(np.int64)
         mk = masks[e0:e1].astype(np.uint64)  # [entries, 2]
         first = np.array([pref_slots(x)[0] for x in pg], dtype=np.int64)
-        assert np.all(np.diff(first) > 0), "column entries must be in ascending slot order"
+        # half of every entry: 0 for the 128-row route; entries 4i, 4i+1 of
+        # the 64-row route serve rows 0..63, entries 4i+2, 4i+3 rows 64..127
+        ehalf = (np.arange(e1 - e0) % 4) // 2 if route else np.zeros(e1 - e0, np.int64)
+        if route:
+            assert which == 0 and n_own == 8 and (e1 - e0) % 4 == 0
+            for hf in (0, 1):
+                live = (ehalf == hf) & ((mk[:, 0] | mk[:, 1]) != 0)
+                assert np.all(np.diff(first[live]) > 0), "each half's entries in ascending slot order"
+        else:
+            assert np.all(np.diff(first) > 0), "column entries must be in ascending slot order"
         col_slot = np.stack([pref_slots(x) for x in pg]) if pg.size else np.zeros((0, 16), np.int64)
         for r in range(128):
             c = int(codes[r])
@@ -99,6 +110,11 @@ def _covered(p, pl, which, head_filter=None, row_filter=None):
                 continue
             assert c < 8 and own_group[slot] >= 0
             bits = ((mk[:, c // 4, None] >> (np.uint64(16 * (c % 4)) + bits16)) & np.uint64(1)).astype(bool)
+            if route:
+                # a row of half r // 64 sees only its half's entries, and the
+                # other half's entries carry no bit of its segment (so that a
+                # kernel running every entry against all rows stays exact)
+                assert not bits[ehalf != r // 64].any()
             cols = col_slot[bits]
             assert np.all(cols < col_slots)
             for col in cols.tolist():
@@ -118,18 +134,22 @@ def _split_pages(pl, which):
 
 @pytest.mark.parametrize("name", TINY)
 @pytest.mark.parametrize("which", [0, 1])
-@pytest.mark.parametrize("pack", ["best", "split"])
+@pytest.mark.parametrize("pack", ["best", "split", "route64"])
 def test_coverage_invariant_tiny(name, which, pack, monkeypatch):
     """Every allowed pair exactly once, on exactly one owned row; with the
     group-split packing forced, pages shared by several work items (each
-    owning the rows of its group) are covered exactly once as well."""
+    owning the rows of its group) are covered exactly once as well; with the
+    64-row route forced, each half of a tile over its own list."""
     p = W.make_problem(name)
-    if pack == "split":
-        monkeypatch.setenv("SPATTN_PLAN_PACK", "split")
+    if pack != "best":
+        monkeypatch.setenv("SPATTN_PLAN_PACK", pack)
     pl = sp.Plan.from_problem(p)
     monkeypatch.delenv("SPATTN_PLAN_PACK", raising=False)
     if pack == "split" and name == "tiny_svg2":
         assert _split_pages(pl, which) > 0  # the clustered layout does split pages
+    if pack == "route64":
+        routed = pl.work(which)[0][:, 28]
+        assert np.all(routed == 1) if which == 0 else np.all(routed == 0)
     pairs, owned = _covered(p, pl, which)
     assert all(v == 1 for v in pairs.values()), "a pair is computed by two owned rows"
     own_group = p.q_group if which == 0 else p.kv_group
