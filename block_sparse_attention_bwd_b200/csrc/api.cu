@@ -152,6 +152,7 @@ TileArgs tile_args(const spattn_plan_s* P, const WorkList& w, int64_t own_slots,
   a.kv_group = P->heads / P->kv_heads;
   // entry head offsets exist only under grouped-query attention (else all 0)
   a.col_heads = P->kv_heads == P->heads ? nullptr : w.d_heads;
+  a.route64 = w.route64;
   return a;
 }
 

@@ -501,6 +501,7 @@ int device_replan(spattn_plan_s* P, const int64_t* row_ptr, const int32_t* kv_gr
                       st>>>(la[pass]);
     if (cudaGetLastError() != cudaSuccess) return SPATTN_ERR_CUDA;
     wl.n_work = n_work;
+    wl.route64 = false;  // the templates are 128-row items
     wl.n_entries_dev = total;
     wl.physical_pairs = static_cast<int64_t>(kTilePages * kPageRows) * kPageRows * total * copies;
   }

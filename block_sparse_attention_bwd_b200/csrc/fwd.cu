@@ -57,7 +57,9 @@ constexpr float kRescaleThreshold = 8.0f;
 // threads (warp w reaches TMEM lanes 32*(w%4) .. 32*(w%4)+31).
 constexpr int kFwdThreads = 192;
 
-template <int D, bool F8>
+// ROUTE: the form that reads each item's route flag (the 64-row route of
+// Work::halves); without it every item runs as 128 rows over its whole list.
+template <int D, bool F8, bool ROUTE>
 __global__ void __launch_bounds__(kFwdThreads, 2)
     fwd_kernel(const __grid_constant__ TmaPages tm_q, const __grid_constant__ TmaPages tm_k,
                const __grid_constant__ TmaPages tm_v, const int32_t* __restrict__ work,
@@ -93,7 +95,7 @@ __global__ void __launch_bounds__(kFwdThreads, 2)
   const int n_cols = wk.e1 - wk.e0;
   const int n_steps = (n_cols + NP - 1) / NP;
   // 64-row route: every step holds two pages per half (a list of whole steps)
-  const bool halves = wk.halves() && (n_cols % NP) == 0;
+  const bool halves = ROUTE && wk.halves() && (n_cols % NP) == 0;
   const int warp = warp_id(), lane = lane_id();
 
   if (threadIdx.x == 0) {
@@ -421,18 +423,27 @@ __global__ void fill_kernel(const int32_t* __restrict__ fill, int64_t n_bh, int6
   }
 }
 
+template <int D, bool F8, bool ROUTE>
+cudaError_t launch_fwd_r(const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
+                         __nv_bfloat16* o, float* lse, const float* q_descale, const float* k_descale,
+                         cudaStream_t st) {
+  using C = FwdCfg<D, F8>;
+  cudaError_t e =
+      cudaFuncSetAttribute(fwd_kernel<D, F8, ROUTE>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+  if (e != cudaSuccess) return e;
+  if (a.n_work == 0) return cudaSuccess;
+  fwd_kernel<D, F8, ROUTE><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
+      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.heads, a.kv_group, q_descale,
+      k_descale, a.err);
+  return cudaGetLastError();
+}
+
 template <int D, bool F8>
 cudaError_t launch_fwd_t(const TmaPages& tq, const TmaPages& tk, const TmaPages& tv, const TileArgs& a,
                          __nv_bfloat16* o, float* lse, const float* q_descale, const float* k_descale,
                          cudaStream_t st) {
-  using C = FwdCfg<D, F8>;
-  cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-  if (e != cudaSuccess) return e;
-  if (a.n_work == 0) return cudaSuccess;
-  fwd_kernel<D, F8><<<static_cast<unsigned>(a.n_work), kFwdThreads, C::kSmem, st>>>(
-      tq, tk, tv, a.work, a.pages, a.masks, o, lse, a.own_slots, a.scale * kLog2e, a.heads, a.kv_group, q_descale,
-      k_descale, a.err);
-  return cudaGetLastError();
+  return a.route64 ? launch_fwd_r<D, F8, true>(tq, tk, tv, a, o, lse, q_descale, k_descale, st)
+                   : launch_fwd_r<D, F8, false>(tq, tk, tv, a, o, lse, q_descale, k_descale, st);
 }
 
 }  // namespace

@@ -45,6 +45,9 @@ struct TileArgs {
   // pass, entry e's column head is the item's first query head + col_heads[e].
   int heads = 1, kv_heads = 1, kv_group = 1;
   const uint16_t* col_heads = nullptr;
+  // some query-owned item takes the 64-row route (the forward then runs the
+  // kernel form that reads the route flag of each item)
+  bool route64 = false;
 };
 
 // K1: O, LSE for every query-owned work item.

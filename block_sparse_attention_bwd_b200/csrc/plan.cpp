@@ -865,6 +865,8 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   wl.work.swap(all);
   wl.n_work = per_copy * batch_copies;
   wl.physical_pairs *= batch_copies;
+  wl.route64 = false;
+  for (size_t i = 28; i < wl.work.size(); i += kWorkWords) wl.route64 = wl.route64 || wl.work[i] != 0;
   return SPATTN_OK;
 }
 

@@ -66,6 +66,7 @@ struct WorkList {
   std::vector<uint16_t> heads;
   uint16_t* d_heads = nullptr;
   int64_t n_work = 0;
+  bool route64 = false;          // some item takes the 64-row route (word 28)
   int64_t physical_pairs = 0;    // one batch
   int32_t* d_work = nullptr;
   int32_t* d_pages = nullptr;
