@@ -93,6 +93,27 @@ def test_device_replan_parity_tiny(name):
     check_tiny(q, t, out, 1)
 
 
+def test_device_replan_of_a_routed_plan(monkeypatch):
+    """A host plan whose query-owned items take the 64-row route, re-planned
+    on the device: the new items are 128-row (route word 0, the kernel form
+    without the route), and the forward and backward match the oracle."""
+    from test_gpu_parity import check_tiny, run_gpu
+
+    p = W.make_problem("tiny_vsa")
+    monkeypatch.setenv("SPATTN_PLAN_PACK", "route64")
+    pl = sp.Plan.from_problem(p)
+    monkeypatch.delenv("SPATTN_PLAN_PACK")
+    assert (pl.work(0)[0][:, 28] == 1).all()
+    row_ptr, cols = _graph_variant(p, 13)
+    _replan(pl, row_ptr, cols)
+    assert (pl.work(0)[0][:, 28] == 0).all()
+    assert _items(pl, 0) == _items(_host_slot_plan(p, row_ptr, cols, monkeypatch), 0)
+    q = W.Problem(p.name, p.batch, p.heads, p.head_dim, p.q_group, p.kv_group, p.n_q_groups, p.n_kv_groups, row_ptr,
+                  cols, p.seed_base)
+    t, out, _ = run_gpu(q, pl=pl)
+    check_tiny(q, t, out, 1)
+
+
 @pytest.mark.parametrize("name,batch", [("tiny_gqa", 2), ("tiny_mqa", 1), ("tiny_bgraph", 2)])
 def test_device_replan_grouped_heads_and_batch_graphs(name, batch, monkeypatch):
     """Grouped-query attention (key-owned entries carry their query-head
