@@ -137,8 +137,10 @@ int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_p
  * planner groups 64-slot blocks into owned tiles in two ways, slot order and
  * grouping by the overlap of the blocks' column lists, and keeps the one
  * that computes fewer physical pairs; SPATTN_PLAN_PACK=slot or =similar
- * forces one of them.  Work items of a head run longest column list
- * first.) */
+ * forces one of them.  The query-owned pass may instead take the 64-row
+ * route (work word 28, see spattn_plan_work) where a cost model of the
+ * forward and dQ steps favours it; SPATTN_PLAN_PACK=route64 forces it.
+ * Work items of a head run longest column list first.) */
 
 /* Re-plan for a new sparse graph over the plan's layout, on the GPU.
  * Dynamic block selection (VSA-style graphs, one of the layouts the KPage
