@@ -209,6 +209,32 @@ def test_page_lists_and_counts_large_sampled(name):
         assert got == exp
 
 
+@pytest.mark.parametrize("name", ["vsa", "partial"])
+def test_route64_large_sampled(name, monkeypatch):
+    """The 64-row route forced on a full-size layout: every query-owned item
+    is routed with whole 4-entry steps, the physical-pair count is 64 rows x
+    16 columns per entry, and sampled query rows of one head see exactly
+    their allowed keys (through their own half's entries only)."""
+    p = W.make_problem(name)
+    monkeypatch.setenv("SPATTN_PLAN_PACK", "route64")
+    pl = sp.Plan.from_problem(p)
+    monkeypatch.delenv("SPATTN_PLAN_PACK")
+    work, pages, _ = pl.work(0)
+    assert (work[:, 28] == 1).all() and ((work[:, 3] - work[:, 2]) % 4 == 0).all()
+    st = pl.stats()
+    assert st["physical_pairs_fwd"] == 64 * 16 * int((work[:, 3] - work[:, 2]).sum())
+    assert st["physical_pairs_fwd"] >= st["useful_pairs"]
+    rng = np.random.default_rng(23)
+    h = int(rng.integers(p.heads))
+    A = _allowed(p, h)
+    rows = set(rng.integers(0, p.q_slots, size=6).tolist())
+    pairs, _ = _covered(p, pl, 0, head_filter={h}, row_filter=rows)
+    assert all(v == 1 for v in pairs.values())
+    M = oracle.token_mask(p.q_group, p.kv_group, A, np.array(sorted(rows)))
+    for k, i in enumerate(sorted(rows)):
+        assert sorted(j for (hh, ii, j) in pairs if ii == i) == np.nonzero(M[k])[0].tolist()
+
+
 @pytest.mark.parametrize("name", ["partial", "svg2"])
 def test_plan_independent_of_thread_count(name, monkeypatch):
     p = W.with_heads(W.make_problem(name), 5)
