@@ -37,6 +37,7 @@
 #include <queue>
 #include <thread>
 #include <tuple>
+#include <unordered_map>
 
 namespace spattn {
 
@@ -770,6 +771,47 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   // takes units t, t + n, ...), then the parts are joined in unit order, so
   // the result does not depend on the number of threads.
   std::vector<WorkList> part(n_units);
+  // Units whose column sources are the same graph rows get the same list
+  // (every head of a layout whose heads share one graph, as the STA-style
+  // windows do): it is built for the first such unit and copied, with the
+  // owned head rewritten.  SPATTN_PLAN_DEDUP=0 builds every unit (the plans
+  // are identical; tests compare them).
+  std::vector<int32_t> same_as(n_units, -1);
+  const char* dedup_env = std::getenv("SPATTN_PLAN_DEDUP");
+  if (!(dedup_env && std::strcmp(dedup_env, "0") == 0)) {
+    auto same_rows = [&](const std::vector<int64_t>& a, const std::vector<int64_t>& b) {
+      if (a.size() != b.size()) return false;
+      for (size_t j = 0; j < a.size(); ++j)
+        for (int32_t g = 0; g < adj.n_src; ++g) {
+          const int64_t ra = a[j] * adj.n_src + g, rb = b[j] * adj.n_src + g;
+          const int64_t na = adj.ptr[ra + 1] - adj.ptr[ra];
+          if (na != adj.ptr[rb + 1] - adj.ptr[rb] ||
+              !std::equal(adj.dst.begin() + adj.ptr[ra], adj.dst.begin() + adj.ptr[ra + 1], adj.dst.begin() + adj.ptr[rb]))
+            return false;
+        }
+      return true;
+    };
+    std::unordered_map<uint64_t, std::vector<int32_t>> seen;
+    for (int32_t u = 0; u < n_units; ++u) {
+      const std::vector<int64_t> src = src_heads(u);
+      uint64_t h = 1469598103934665603ull;  // FNV-1a over the rows' lengths and entries
+      auto mix = [&](uint64_t x) { h = (h ^ x) * 1099511628211ull; };
+      mix(src.size());
+      for (int64_t sh : src)
+        for (int32_t g = 0; g < adj.n_src; ++g) {
+          const int64_t r = sh * adj.n_src + g;
+          mix(static_cast<uint64_t>(adj.ptr[r + 1] - adj.ptr[r]));
+          for (int64_t e = adj.ptr[r]; e < adj.ptr[r + 1]; ++e) mix(static_cast<uint32_t>(adj.dst[e]));
+        }
+      auto& cand = seen[h];
+      for (int32_t c : cand)
+        if (same_rows(src_heads(c), src)) {
+          same_as[u] = c;
+          break;
+        }
+      if (same_as[u] < 0) cand.push_back(u);
+    }
+  }
   // all hardware threads, unless SPATTN_PLAN_THREADS (>= 1) asks for fewer or more
   int want = static_cast<int>(std::thread::hardware_concurrency());
   if (const char* env = std::getenv("SPATTN_PLAN_THREADS")) want = std::max(1, std::atoi(env));
@@ -780,6 +822,7 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
       std::vector<int64_t> touched;
       std::vector<uint64_t> acc;
       for (int32_t u = t; u < n_units; u += n_threads) {
+        if (same_as[u] >= 0) continue;
         const std::vector<int64_t> src = src_heads(u);
         acc.assign(static_cast<size_t>(col.n_pages) * src.size() * kMaskWords, 0);
         // Per unit, the packing with fewer physical pairs (then fewer items).
@@ -829,6 +872,15 @@ int build_worklist(const Side& own, const Side& col, const Adjacency& adj, int32
   }
   for (char f : failed)
     if (f) return SPATTN_ERR_OOM;
+  try {
+    for (int32_t u = 0; u < n_units; ++u) {
+      if (same_as[u] < 0) continue;
+      part[u] = part[same_as[u]];
+      for (size_t i = 0; i < part[u].work.size(); i += kWorkWords) part[u].work[i] = u;
+    }
+  } catch (...) {
+    return SPATTN_ERR_OOM;
+  }
   size_t n_entries = 0;
   for (const auto& pt : part) n_entries += pt.pages.size();
   if (n_entries > static_cast<size_t>(INT32_MAX)) return SPATTN_ERR_UNSUPPORTED;

@@ -133,6 +133,8 @@ typedef struct {
 int spattn_plan(const spattn_layout* layout, const spattn_graph* graph, spattn_plan_t* out);
 /* (Heads are planned in parallel on all hardware threads; the environment
  * variable SPATTN_PLAN_THREADS, if set to n >= 1, uses n threads instead.
+ * Heads whose graph rows are identical are planned once and copied
+ * (SPATTN_PLAN_DEDUP=0 plans every head; the result is the same).
  * The plan is identical for every thread count.  Per head and pass, the
  * planner groups 64-slot blocks into owned tiles in two ways, slot order and
  * grouping by the overlap of the blocks' column lists, and keeps the one

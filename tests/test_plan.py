@@ -235,6 +235,24 @@ def test_route64_large_sampled(name, monkeypatch):
         assert sorted(j for (hh, ii, j) in pairs if ii == i) == np.nonzero(M[k])[0].tolist()
 
 
+@pytest.mark.parametrize("name,batch", [("partial", 1), ("tiny_gqa", 2), ("tiny_bgraph", 2), ("tiny_vsa", 1)])
+def test_plan_dedup_of_identical_heads(name, batch, monkeypatch):
+    """Heads with the same graph rows are planned once and copied: the
+    plan equals, word for word, the plan that builds every head."""
+    p = W.make_problem(name)
+    plans = []
+    for dedup in ("1", "0"):
+        monkeypatch.setenv("SPATTN_PLAN_DEDUP", dedup)
+        pl = sp.Plan.from_problem(p, batch=batch)
+        plans.append(([np.array(x, copy=True) for w in (0, 1) for x in pl.work(w)]
+                      + [np.array(pl.entry_heads(w), copy=True) for w in (0, 1)], pl.stats()))
+    monkeypatch.delenv("SPATTN_PLAN_DEDUP")
+    (a, sa), (b, sb) = plans
+    assert all(np.array_equal(x, y) for x, y in zip(a, b))
+    for k in ("useful_pairs", "physical_pairs_fwd", "physical_pairs_dkdv", "n_work_fwd", "n_work_dkdv"):
+        assert sa[k] == sb[k], k
+
+
 @pytest.mark.parametrize("name", ["partial", "svg2"])
 def test_plan_independent_of_thread_count(name, monkeypatch):
     p = W.with_heads(W.make_problem(name), 5)
