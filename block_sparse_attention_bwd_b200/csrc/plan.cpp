@@ -1131,23 +1131,47 @@ int build_plan(const spattn_layout* L, const spattn_graph* G, spattn_plan_s* P) 
   const int32_t copies = L->batch / gb;  // batch entries that share each graph
   P->useful_pairs = useful * copies;
 
-  // query-owned pass: unit = graph head (its own graph rows)
-  st = build_worklist(P->q, P->k, P->fwd_adj, GH, L->heads, copies,
-                      [](int32_t u) { return std::vector<int64_t>{u}; }, true, P->wq);
-  if (st) return st;
   // key-owned pass: unit = K/V head of a graph batch; its columns are the
-  // transposed rows of the query heads of its group (head offset j)
+  // transposed rows of the query heads of its group (head offset j).  It
+  // only reads the layout and its own adjacency, so it runs on a thread of
+  // its own while this thread builds the query-owned pass (after it, if no
+  // thread can be created).
   const int32_t grp = L->heads / kv_heads;
   const int32_t H = L->heads;
-  st = build_worklist(P->k, P->q, P->bwd_adj, gb * kv_heads, kv_heads, copies,
-                      [=](int32_t u) {
-                        std::vector<int64_t> v(grp);
-                        for (int32_t j = 0; j < grp; ++j)
-                          v[j] = static_cast<int64_t>(u / kv_heads) * H + (u % kv_heads) * grp + j;
-                        return v;
-                      },
-                      false, P->wk);
+  const int32_t n_kv_units = gb * kv_heads;
+  int st_k = SPATTN_OK;
+  auto key_pass = [&]() {
+    try {
+      st_k = build_worklist(P->k, P->q, P->bwd_adj, n_kv_units, kv_heads, copies,
+                            [=](int32_t u) {
+                              std::vector<int64_t> v(grp);
+                              for (int32_t j = 0; j < grp; ++j)
+                                v[j] = static_cast<int64_t>(u / kv_heads) * H + (u % kv_heads) * grp + j;
+                              return v;
+                            },
+                            false, P->wk);
+    } catch (...) {
+      st_k = SPATTN_ERR_OOM;
+    }
+  };
+  std::thread key_thread;
+  bool key_threaded = false;
+  try {
+    key_thread = std::thread(key_pass);
+    key_threaded = true;
+  } catch (...) {
+  }
+  // query-owned pass: unit = graph head (its own graph rows)
+  try {
+    st = build_worklist(P->q, P->k, P->fwd_adj, GH, L->heads, copies,
+                        [](int32_t u) { return std::vector<int64_t>{u}; }, true, P->wq);
+  } catch (...) {
+    st = SPATTN_ERR_OOM;
+  }
+  if (key_threaded) key_thread.join();
+  else key_pass();
   if (st) return st;
+  if (st_k) return st_k;
 
   fill_list(P->q, P->q_fill);
   fill_list(P->k, P->k_fill);
