@@ -410,11 +410,6 @@ std::vector<std::vector<int32_t>> pack_similar(const Side& col, const Adjacency&
   return tiles;
 }
 
-// Work items of one head for one pass; work words use bh = head (batch 0).
-// Work items of one unit for one pass.  A unit is one owned head (w[0]
-// before batch replication) whose columns come from the adjacency rows of the
-// graph heads src_heads[j]: one for the query-owned pass, the query heads of
-// a K/V head's group for the key-owned pass (entries carry j).
 // Column entries of one list, in slot order, from the masks accumulated in
 // `acc` for the (head offset, page) keys of `touched` (sorted); the keys' acc
 // words are cleared on the way.  Up to four consecutive pages whose attended
@@ -471,6 +466,11 @@ void append_entries(const Side& col, bool strided, std::vector<uint64_t>& acc, c
   }
 }
 
+// Work items of one unit for one pass (work words use bh = the unit, batch
+// 0).  A unit is one owned head (w[0] before batch replication) whose
+// columns come from the adjacency rows of the graph heads src_heads[j]: one
+// for the query-owned pass, the query heads of a K/V head's group for the
+// key-owned pass (entries carry j).
 void build_head(const Side& own, const Side& col, const Adjacency& adj, int32_t unit,
                 const std::vector<int64_t>& src_heads, const std::vector<std::vector<int32_t>>& tiles, WorkList& wl,
                 std::vector<uint64_t>& acc, std::vector<int64_t>& touched,
