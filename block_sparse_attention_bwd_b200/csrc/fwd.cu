@@ -19,6 +19,12 @@
 //               masks, running max with lazy rescaling, P in bf16 to TMEM,
 //               and the epilogue (O / l, LSE in natural log).
 // S is double-buffered, so the MMA of step c+1 overlaps the softmax of c.
+//
+// 64-row route (the kernel form with ROUTE, for work lists that hold routed
+// items): rows 0..63 and 64..127 each run over their own two pages of every
+// step, as two M = 64 products written to the same 32 columns at TMEM lane
+// offsets 0 and 16 (row r of half h at lane 16h + r % 16 + 32 (r / 16)),
+// and two M = 64 P.V products that read P from those lanes.
 #include "kernels.cuh"
 #include "tile.cuh"
 
