@@ -1,8 +1,9 @@
 """FP8 (E4M3) quantisation of Q and K for the FP8 forward — TEST INFRASTRUCTURE ONLY.
 
 The FP8 forward variant computes S = Q K^T on the tensor core from E4M3 codes
-(the low-precision line of work the KPage survey lists next to the method:
-quantised Q / K, exact attention otherwise).  What it must reach exactly is
+(the quantised-attention line of work, e.g. SageAttention2 in the related-paper
+list of the scifaro.com related-papers page for arXiv 2411.10958: quantised
+Q / K, exact attention otherwise).  What it must reach exactly is
 masked softmax attention of the *dequantised* inputs, so the oracle is
 
     q_hat = decode(q8) * q_descale[b, h],   k_hat = decode(k8) * k_descale[b, h]
